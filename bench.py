@@ -1,0 +1,490 @@
+"""Benchmark of the FP8 paged decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gqa|ragged|long] [--no-bf16] [--no-cpu-baseline]
+
+A step is one pass of the whole hot path over one decode batch:
+kvq_append (the new token of every sequence) -> kvq_validate (page tags ->
+abort mask) -> kvq_decode (split-KV attention + log-sum-exp combine).  The
+default workload is the GQA decode batch: 32 sequences x 8,192 tokens, page
+16, 64 query / 8 KV heads, head_dim 128, E4M3 cache with per-head scales.
+The cache (537 MB of codes) is larger than L2, so no flush is needed.
+
+`value` is KV GB/s: cache bytes one decode step reads / device time per step
+(CUDA events, steps replayed from a CUDA graph, max over ranks).  N > 1 runs
+N independent replicas (one per GPU, no collective on the data path) and
+reports the aggregate.  `--impl reference` times the CPU oracle on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 paged decode attention: KV GB/s (% of HBM peak) and decode tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gqa")
+    ap.add_argument("--num-ctas", type=int, default=0)
+    ap.add_argument("--no-bf16", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="keep only the first N sequences (smaller case for profiling)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.ok = False
+        self.samples = []
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report nothing rather than guess
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.stop = False
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop = True
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable" if not self.ok else "no samples"}
+        mhz = [s for s, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = sorted(n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# timing helpers
+# ---------------------------------------------------------------------------
+def time_graph(graph, K, stream):
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / K
+
+
+def capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def dist_setup(args):
+    if args.gpus <= 1 and "WORLD_SIZE" not in os.environ:
+        return 0, 1, 0
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample of the same workload)
+# ---------------------------------------------------------------------------
+def oracle_sample(spec_name, n_groups, seed=0):
+    """Oracle cache for the first (sequence, KV head) groups of the workload.
+
+    Returns (step, kv_bytes, description): step() runs the oracle's
+    append (new tokens) + validate + decode (the groups' query heads)."""
+    import oracle
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    full = W.spec_by_name(spec_name, seed)
+    H, G = full.num_kv_heads, full.group
+    nseq = min(full.B, -(-n_groups // H))
+    n_groups = min(n_groups, nseq * H)
+    spec = W.Spec(full.name + "_sample", list(full.seq_lens)[:nseq], full.page_size,
+                  full.num_q_heads, H, full.head_dim_k, full.head_dim_v, v_alias=full.v_alias,
+                  kv_dtype=full.kv_dtype, scale_mode=full.scale_mode, outlier_p=full.outlier_p,
+                  n_stale=0, sm_scale=full.sm_scale)
+    wl = W.make_workload(spec, seed=seed, device="cpu")
+    s = spec
+    P, ps = wl.num_pages, s.page_size
+    fp8 = s.kv_dtype == W.FP8
+    el = np.uint8 if fp8 else np.uint16
+    kp = np.zeros((P, H, ps, s.head_dim_k), el)
+    vp = None if s.v_alias else np.zeros((P, H, ps, s.head_dim_v), el)
+    mode = {W.SCALE_TENSOR: 0, W.SCALE_HEAD: 1, W.SCALE_TOKEN: 2}[s.scale_mode]
+    if mode == 2:
+        ks = np.ones((P, H, ps), np.float32)
+        vs = None if s.v_alias else np.ones((P, H, ps), np.float32)
+    else:
+        n = 1 if mode == 0 else H
+        ks, vs = np.ones(n, np.float32), (None if s.v_alias else np.ones(n, np.float32))
+    oc = oracle.Cache(oracle.FP8 if fp8 else oracle.BF16, mode, P, ps, H, s.head_dim_k,
+                      s.head_dim_v, kp, vp, ks, vs, wl.page_tags.copy())
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    hist = [(bits(k), None if v is None else bits(v), sl) for k, v, sl in wl.hist_chunks()]
+    if fp8 and mode != 2:
+        oc.k_scale[:] = oracle.scales(np.concatenate([h[0] for h in hist]), mode == 1)
+        if vs is not None:
+            oc.v_scale[:] = oracle.scales(np.concatenate([h[1] for h in hist]), mode == 1)
+    for k, v, sl in hist:
+        oracle.append(oc, k, v, sl)
+    del hist
+    kn, vn, slots = wl.new_tokens()
+    knb, vnb = bits(kn), (None if vn is None else bits(vn))
+    qb = bits(wl.q())
+    rows = np.array([(g // H) * s.num_q_heads + (g % H) * G + i
+                     for g in range(n_groups) for i in range(G)], np.int32)
+    row_bytes = wl.kv_row_bytes + (4 if (fp8 and mode == 2) else 0)
+    kv = sum(int(wl.seq_lens[g // H]) for g in range(n_groups)) * row_bytes
+
+    def step():
+        oracle.append(oc, knb, vnb, slots)
+        m = oracle.validate(oc.page_tags, wl.block_table, wl.expected_tags, wl.seq_lens, ps)
+        oracle.decode(oc, qb, wl.block_table, wl.seq_lens, m, wl.sm_scale, rows=rows)
+
+    desc = (f"{n_groups} (sequence, KV head) groups = {rows.size} query rows of the {full.name} "
+            f"workload ({kv / 1e6:.1f} MB of cache), step = append + validate + decode")
+    return step, kv, desc
+
+
+def cpu_baseline(spec_name, budget_s, seed=0):
+    """The oracle as it stands, timed on the host cores on a sample of the
+    workload sized to about budget_s seconds (one step)."""
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    full = W.spec_by_name(spec_name, seed)
+    step1, _, _ = oracle_sample(spec_name, 1, seed)
+    t0 = time.perf_counter()
+    step1()
+    t1 = time.perf_counter() - t0
+    n = max(1, min(full.B * full.num_kv_heads, int(budget_s / max(t1, 1e-6))))
+    step, kv, desc = oracle_sample(spec_name, n, seed)
+    t0 = time.perf_counter()
+    step()
+    dt = time.perf_counter() - t0
+    return {"value": kv / dt / 1e9, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle", "sample": desc, "seconds": dt}
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the oracle as it stands
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    # per-step budget so that warm-up + steps end in a few minutes
+    per_step = max(0.02, 150.0 / max(1, args.steps + args.warmup))
+    step1, _, _ = oracle_sample(args.workload, 1)
+    t0 = time.perf_counter()
+    step1()
+    t1 = time.perf_counter() - t0
+    n = max(1, int(per_step / max(t1, 1e-6)))
+    step, kv, desc = oracle_sample(args.workload, n)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    cores = len(os.sched_getaffinity(0))
+    value = kv / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(args.workload), "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_desc(name, seqs=0):
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    s = W.spec_by_name(name)
+    if seqs:
+        s.seq_lens = list(s.seq_lens)[:seqs]
+    lens = sorted(set(s.seq_lens))
+    ltxt = f"{s.B} seq x {lens[0]} tok" if len(lens) == 1 else f"{s.B} seq, {min(lens)}..{max(lens)} tok"
+    return (f"{name}: {ltxt}, page {s.page_size}, {s.num_q_heads}q/{s.num_kv_heads}kv heads, "
+            f"d{s.head_dim_k}/{s.head_dim_v}, {s.kv_dtype} {s.scale_mode} scales")
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    rank, world, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import fp8_kv_paged_kvq_b200 as kvq
+    from fp8_kv_paged_kvq_b200 import build as kvq_build
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch
+    if rank == 0:
+        kvq_build.build()
+    barrier(world) if world > 1 else None
+    kvq.lib()
+
+    spec = W.spec_by_name(args.workload)
+    if args.seqs:
+        spec.seq_lens = list(spec.seq_lens)[: args.seqs]
+    wl = W.make_workload(spec, seed=0, device=dev)
+    db = DecodeBatch(wl, device=dev, num_ctas=args.num_ctas)
+    db.prefill()
+    torch.cuda.synchronize()
+    kv_bytes = wl.kv_bytes_read()
+    s = spec
+    alg_bytes = (kv_bytes + s.B * s.num_q_heads * s.head_dim_k * 2          # q
+                 + int(np.ceil(wl.seq_lens / s.page_size).sum()) * 4        # block table
+                 + s.B * s.num_q_heads * (s.head_dim_v + 1) * 4)            # out + lse
+    stream = torch.cuda.Stream(device=dev)
+    hbm, hbm_kind = peaks()
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            db.step(check_tags=True, stream=stream)
+        torch.cuda.synchronize()
+        g_step = capture(lambda: db.step(check_tags=True, stream=stream), stream)
+        g_nochk = capture(lambda: db.step(check_tags=False, stream=stream), stream)
+        g_dec = capture(lambda: db.decode(use_abort=True, stream=stream), stream)
+        for g in (g_step, g_nochk, g_dec):
+            for _ in range(3):
+                g.replay()
+        torch.cuda.synchronize()
+
+        # ---- the timed region: K steps ----
+        barrier(world)
+        sampler = ClockSampler(local)
+        with sampler:
+            ms_step = time_graph(g_step, args.steps, stream)
+        barrier(world)
+        ms_step = max_over_ranks(ms_step, world)
+        # dominant kernel (kvq_decode: split-KV kernel + combine), same data
+        ms_dec = max_over_ranks(time_graph(g_dec, args.steps, stream), world)
+        ms_nochk = max_over_ranks(time_graph(g_nochk, args.steps, stream), world)
+    assert kvq.device_error() == 0, "device-side wait timed out"
+
+    # ---- e2e through the public API with host buffers ----
+    e2e = run_e2e(db, args, stream, kv_bytes, world)
+
+    # ---- BF16 cache, same shapes ----
+    bf16 = None
+    if not args.no_bf16 and s.kv_dtype == W.FP8 and not s.v_alias:
+        del g_step, g_nochk, g_dec
+        bf16 = run_bf16(wl, args, stream, world, dev)
+
+    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    achieved = alg_bytes / (ms_dec * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16 mma / f32 accumulate (e4m3 cache)",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(args.workload, args.seqs),
+                   "step": "kvq_append + kvq_validate + kvq_decode (split-KV + LSE combine)",
+                   "l2": f"inputs exceed L2: {kv_bytes / 1e6:.0f} MB of cache read per step",
+                   "timing": "CUDA graph replay, CUDA events, max over ranks",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "decode_tokens_per_s": world * s.B / (ms_step * 1e-3),
+        "hbm_frac_of_step": value / world / hbm,
+        "validate_overhead_pct": 100.0 * (ms_step - ms_nochk) / ms_nochk,
+        "ms_per_step_without_validation": ms_nochk,
+        "roofline": {"bound": "hbm", "kernel": "kvq_decode (gqa_decode_kernel + lse_combine_kernel)",
+                     "achieved": achieved, "peak": hbm, "peak_kind": hbm_kind, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "algorithmic_bytes_per_launch": alg_bytes, "ms_per_launch": ms_dec},
+        "gpu_launches": 4 * args.steps,
+        "clocks": sampler.summary(),
+        "e2e": e2e,
+    }
+    if bf16:
+        line["bf16_same_shape"] = bf16
+        line["fp8_vs_bf16_step_time"] = ms_step / bf16["ms_per_step"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=10.0)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(db, args, stream, kv_bytes, world):
+    """Same step through the Python API, step inputs copied from pinned host
+    memory and the result read back, every step."""
+    import fp8_kv_paged_kvq_b200 as kvq
+    K = args.e2e_steps
+    host_in = {name: t.detach().cpu().pin_memory() for name, t in
+               (("q", db.q), ("k_new", db.k_new), ("v_new", db.v_new), ("slots", db.new_slots),
+                ("seq_lens", db.seq_lens), ("block_table", db.block_table),
+                ("expected", db.expected)) if t is not None}
+    dev_in = {"q": db.q, "k_new": db.k_new, "v_new": db.v_new, "slots": db.new_slots,
+              "seq_lens": db.seq_lens, "block_table": db.block_table, "expected": db.expected}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    out_h = torch.empty(db.out.shape, dtype=db.out.dtype).pin_memory()
+    lse_h = torch.empty(db.lse.shape, dtype=db.lse.dtype).pin_memory()
+    ab_h = torch.empty(db.abort.shape, dtype=db.abort.dtype).pin_memory()
+    d2h = sum(t.numel() * t.element_size() for t in (out_h, lse_h, ab_h))
+
+    def one():
+        for name, h in host_in.items():
+            dev_in[name].copy_(h, non_blocking=True)
+        db.step(check_tags=True, stream=stream)
+        out_h.copy_(db.out, non_blocking=True)
+        lse_h.copy_(db.lse, non_blocking=True)
+        ab_h.copy_(db.abort, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            one()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / K, world)
+    return {"value": world * kv_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "steps": K, "path": "python binding -> C ABI, eager launches"}
+
+
+def run_bf16(wl_fp8, args, stream, world, dev):
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch
+    db = DecodeBatch(wl_fp8, device=dev, num_ctas=args.num_ctas, kv_dtype=W.BF16)
+    db.prefill()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            db.step(check_tags=True, stream=stream)
+        g = capture(lambda: db.step(check_tags=True, stream=stream), stream)
+        gd = capture(lambda: db.decode(use_abort=True, stream=stream), stream)
+        for _ in range(3):
+            g.replay()
+            gd.replay()
+        barrier(world)
+        ms = max_over_ranks(time_graph(g, args.steps, stream), world)
+        msd = max_over_ranks(time_graph(gd, args.steps, stream), world)
+    kv = 2 * wl_fp8.kv_bytes_read()
+    hbm, _ = peaks()
+    res = {"ms_per_step": ms, "kv_gbs": world * kv / (ms * 1e-3) / 1e9,
+           "decode_ms_per_launch": msd, "decode_kv_gbs": kv / (msd * 1e-3) / 1e9,
+           "decode_frac_of_hbm": kv / (msd * 1e-3) / 1e9 / hbm,
+           "decode_tokens_per_s": world * wl_fp8.B / (ms * 1e-3)}
+    del g, gd, db
+    torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,53 @@
+// Decode-path declarations internal to libkvq (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+struct DecodeArgs {
+  CacheView c;
+  const uint16_t* q;   // bf16 [B][Hq][Dk]
+  int32_t Hq;
+  const int32_t* block_table;
+  int32_t max_pages;
+  const int32_t* seq_lens;
+  int32_t B;
+  const uint8_t* abort_mask;
+  float sm_scale;
+  float* out;
+  float* lse;
+  void* workspace;
+  int32_t num_ctas;
+  cudaStream_t stream;
+};
+
+// Workspace: [B+1] i32 unit prefix | [slots][G] f32 partial lse |
+// [slots][G][Dv] f32 partial outputs, slots = num_ctas + B * Hkv.
+struct WorkspaceLayout {
+  size_t off_pre, off_lse, off_o, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WorkspaceLayout workspace_layout(int32_t B, int32_t Hkv, int32_t G, int32_t Dv,
+                                        int32_t num_ctas) {
+  WorkspaceLayout w;
+  const size_t slots = static_cast<size_t>(num_ctas) + static_cast<size_t>(B) * Hkv;
+  w.off_pre = 0;
+  w.off_lse = align_up(static_cast<size_t>(B + 1) * 4, 256);
+  w.off_o = align_up(w.off_lse + slots * G * 4, 256);
+  w.total = align_up(w.off_o + slots * G * static_cast<size_t>(Dv) * 4, 256);
+  return w;
+}
+
+int gqa_default_ctas(bool fp8, int D, int G, int B);
+void gqa_tma_box(bool fp8, int D, int* box_elems, int* swizzle_bytes);
+cudaError_t launch_gqa_decode(const DecodeArgs& a, const CUtensorMap& km, const CUtensorMap& vm);
+
+}  // namespace kvq

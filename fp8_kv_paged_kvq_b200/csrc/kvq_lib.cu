@@ -1,0 +1,6 @@
+// Single translation unit of libkvq.so: the kernels share one device-side
+// error word, so they are compiled together.
+#include "append.cu"
+#include "validate.cu"
+#include "decode_gqa.cu"
+#include "api.cu"

@@ -1,0 +1,90 @@
+"""A decode batch driven end to end through libkvq: cache set-up, pre-fill,
+and the per-step hot path (append the new token -> validate tags -> decode).
+
+Only library calls touch the data; torch provides device memory and streams.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import (BF16, FP8_E4M3, SCALE_HEAD, SCALE_TENSOR, SCALE_TOKEN, PagedCache, alloc_workspace,
+               amax, append, decode, scale_from_amax, validate)
+from . import workloads as W
+
+_MODE = {W.SCALE_TENSOR: SCALE_TENSOR, W.SCALE_HEAD: SCALE_HEAD, W.SCALE_TOKEN: SCALE_TOKEN}
+
+
+def _dev_i32(a: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int32)).to(device)
+
+
+class DecodeBatch:
+    """Device state of one decode batch built from a seeded workload."""
+
+    def __init__(self, wl: W.Workload, device="cuda", num_ctas: int = 0,
+                 kv_dtype: Optional[str] = None):
+        s = wl.spec
+        self.wl = wl
+        self.device = torch.device(device)
+        dt = kv_dtype or s.kv_dtype
+        self.cache = PagedCache(FP8_E4M3 if dt == W.FP8 else BF16, _MODE[s.scale_mode],
+                                wl.num_pages, s.page_size, s.num_kv_heads, s.head_dim_k,
+                                s.head_dim_v, v_alias=s.v_alias, device=self.device,
+                                tags=_dev_i32(wl.page_tags, "cpu"))
+        self.q = wl.q().to(self.device)
+        self.block_table = _dev_i32(wl.block_table, self.device)
+        self.seq_lens = _dev_i32(wl.seq_lens, self.device)
+        self.expected = _dev_i32(wl.expected_tags, self.device)
+        self.abort = torch.zeros(s.B, dtype=torch.uint8, device=self.device)
+        self.out = torch.empty((s.B, s.num_q_heads, s.head_dim_v), dtype=torch.float32,
+                               device=self.device)
+        self.lse = torch.empty((s.B, s.num_q_heads), dtype=torch.float32, device=self.device)
+        self.num_ctas = num_ctas
+        self.workspace = alloc_workspace(self.cache, s.B, s.num_q_heads, num_ctas, self.device)
+        kn, vn, slots = wl.new_tokens()
+        self.k_new = kn.to(self.device)
+        self.v_new = None if vn is None else vn.to(self.device)
+        self.new_slots = _dev_i32(slots, self.device)
+
+    # -- pre-fill --------------------------------------------------------------
+    def prefill(self, chunk_tokens: Optional[int] = None) -> None:
+        """Scales from the pre-filled tokens (per tensor / per head), then bulk append."""
+        s = self.wl.spec
+        c = self.cache
+        if c.fp8 and s.scale_mode != W.SCALE_TOKEN:
+            per_head = s.scale_mode == W.SCALE_HEAD
+            n = s.num_kv_heads if per_head else 1
+            ak = torch.zeros(n, dtype=torch.float32, device=self.device)
+            av = torch.zeros(n, dtype=torch.float32, device=self.device)
+            for k, v, _ in self.wl.hist_chunks(chunk_tokens):
+                amax(k.to(self.device), per_head, ak)
+                if v is not None:
+                    amax(v.to(self.device), per_head, av)
+            scale_from_amax(ak, out=c.k_scale)
+            if c.v_scale is not None:
+                scale_from_amax(av, out=c.v_scale)
+        for k, v, slots in self.wl.hist_chunks(chunk_tokens):
+            append(c, k.to(self.device), None if v is None else v.to(self.device),
+                   _dev_i32(slots, self.device))
+
+    # -- the hot path of one decode step ----------------------------------------
+    def append_new(self, realloc_pages: Optional[torch.Tensor] = None, stream=None) -> None:
+        append(self.cache, self.k_new, self.v_new, self.new_slots, realloc_pages, stream)
+
+    def validate(self, stream=None) -> torch.Tensor:
+        return validate(self.cache.page_tags, self.block_table, self.expected, self.seq_lens,
+                        self.cache.page_size, self.abort, stream)
+
+    def decode(self, use_abort: bool = True, stream=None):
+        return decode(self.cache, self.q, self.block_table, self.seq_lens,
+                      self.abort if use_abort else None, self.wl.sm_scale, self.out, self.lse,
+                      self.workspace, self.num_ctas, stream)
+
+    def step(self, check_tags: bool = True, stream=None):
+        self.append_new(stream=stream)
+        if check_tags:
+            self.validate(stream)
+        return self.decode(use_abort=check_tags, stream=stream)

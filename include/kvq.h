@@ -1,0 +1,234 @@
+/*
+ * kvq — FP8 (e4m3) paged KV-cache decode path for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libkvq.so.  Plain pointers and sizes only.
+ *
+ * Sources (web pages on one engineering report, cited by page and section):
+ *   [aifeed]  "Cloudflare zrýchľuje inferenciu modelov Kimi a GLM kompresiou
+ *             cache a váh" (aifeed.sk)
+ *   [manulx]  "Công thức của Cloudflare để phục vụ Kimi và GLM: lượng tử hóa
+ *             bộ nhớ đệm KV, nén trọng số, xác minh bộ nhớ đệm" (manulx.blog)
+ *   [remio]   "Cloudflare: Kleinere Modellbereitstellung senkt Speicherbedarf,
+ *             doch Sicherheit wird zum Prüfstein" (remio.ai)
+ *   [lens]    "Cloudflare Workers AI: Kimi および GLM の推論を大規模に最適化する"
+ *             (agentlenshq.com)
+ *
+ * Conventions for every call:
+ *   - All data pointers are DEVICE pointers owned by the caller (the library
+ *     allocates nothing), unless a parameter says "host".
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; no call synchronizes with
+ *     the host except kvq_device_error.
+ *   - Arguments are checked on the host before anything is enqueued; a bad
+ *     argument returns KVQ_ERR_INVALID_ARG (or KVQ_ERR_UNSUPPORTED for a
+ *     shape the kernels do not implement) and enqueues nothing.  A failed
+ *     launch returns KVQ_ERR_CUDA.  Device-resident values (slot ids, page
+ *     ids, sequence lengths) cannot be checked on the host: the kernels clamp
+ *     or skip them as documented below and never read or write out of the
+ *     buffers described here.
+ *   - Calls that share buffers must be ordered on one stream (or by events).
+ *     The intended order within a decode step is
+ *         kvq_append -> kvq_validate -> kvq_decode.
+ *
+ * E4M3: the pages only say "e4m3" ([aifeed] "Dve odlišné úzke miesta v
+ * pamäti GPU"; [lens] "並行性を高めるための KV キャッシュ量子化").  This library
+ * uses the OCP 8-bit floating point E4M3 encoding: bias 7, no infinities,
+ * S.1111.111 = NaN, largest finite 448; conversion rounds to nearest even
+ * and saturates to +-448.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent descriptor */
+  KVQ_ERR_UNSUPPORTED = 2, /* valid but not implemented (head dim, group, page size) */
+  KVQ_ERR_WORKSPACE = 3,   /* workspace missing, too small or misaligned */
+  KVQ_ERR_CUDA = 4         /* a CUDA launch or API call failed */
+} kvq_status;
+
+typedef enum { KVQ_FP8_E4M3 = 0, KVQ_BF16 = 1 } kvq_dtype;
+
+/* Granularity of the FP32 dequantisation scales of an FP8 cache. */
+typedef enum {
+  KVQ_SCALE_TENSOR = 0, /* k_scale[1], v_scale[1] */
+  KVQ_SCALE_HEAD = 1,   /* k_scale[Hkv], v_scale[Hkv] */
+  KVQ_SCALE_TOKEN = 2   /* k_scale[P][Hkv][ps], v_scale[P][Hkv][ps]; written by kvq_append */
+} kvq_scale_mode;
+
+/*
+ * Paged KV cache descriptor.  The cache is split into fixed-size physical
+ * pages shared by all requests, and every page carries a uint32 tag that
+ * changes each time the page is reallocated ([remio] "Sicherheit gemeinsamer
+ * KV-Caches wird zum Produktionsthema"; [manulx] "Bảo vệ bộ nhớ đệm dùng chung").
+ *
+ * Layout (all row-major, device memory owned by the caller):
+ *   k_pages   [P][Hkv][ps][Dk]   FP8: u8 E4M3 codes; BF16: bf16
+ *   v_pages   [P][Hkv][ps][Dv]   or NULL: V is the first Dv dims of each K
+ *                                row (Dv <= Dk) and shares K's scales
+ *   k_scale   FP32, shape per scale_mode (FP8 only; NULL for BF16)
+ *   v_scale   FP32, shape per scale_mode (NULL when v_pages is NULL or BF16)
+ *   page_tags u32 [P]
+ * A token at slot s (0 <= s < P*ps) lives on page s / ps at offset s % ps.
+ * Dequantised value of an FP8 element: fl32(decode(code) * scale).
+ * Base pointers must be 16-byte aligned.
+ */
+typedef struct {
+  int32_t dtype;        /* kvq_dtype */
+  int32_t scale_mode;   /* kvq_scale_mode; ignored for BF16 */
+  int32_t num_pages;    /* P  >= 1 */
+  int32_t page_size;    /* ps >= 1 tokens per page */
+  int32_t num_kv_heads; /* Hkv >= 1 */
+  int32_t head_dim_k;   /* Dk, multiple of 16 */
+  int32_t head_dim_v;   /* Dv, multiple of 16, Dv <= Dk when v_pages == NULL */
+  void* k_pages;
+  void* v_pages;
+  float* k_scale;
+  float* v_scale;
+  uint32_t* page_tags;
+} kvq_cache;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* kvq_status_string(kvq_status status);
+
+/*
+ * Fold max |x| of a BF16 tensor x[T][H][D] into amax_io (FP32): amax_io[0]
+ * over everything (per_head == 0) or amax_io[h] per head (per_head != 0),
+ * as amax_io = max(amax_io, max|x|).  The caller zero-initialises amax_io;
+ * repeated calls over chunks of a tensor accumulate.  NaN elements are
+ * ignored.  Together with kvq_scale_from_amax this gives the per-tensor /
+ * per-head scale amax / 448 that maps the largest element onto the largest
+ * E4M3 code.  (The pages fix no scale granularity; this is the reading that
+ * the per-tensor and per-head workloads use.)
+ * Requires T >= 0, H >= 1, D >= 1 and D % 8 == 0 (16-byte rows).
+ */
+kvq_status kvq_amax(const void* x, int64_t T, int32_t H, int32_t D, int32_t per_head,
+                    float* amax_io, void* stream);
+
+/* scale[i] = fl32(amax[i] / 448) (IEEE division), or 1 where amax[i] is 0
+ * or NaN.  n >= 0.  amax and scale may alias. */
+kvq_status kvq_scale_from_amax(const float* amax, float* scale, int32_t n, void* stream);
+
+/*
+ * Quantize-on-append (write path of the decode pool, where the cache is
+ * stored as E4M3: [aifeed] "Kompresia sa oplatí inde pri vstupe a inde pri
+ * výstupe"; [manulx] "Bộ nhớ đệm KV FP8 tăng gấp đôi dung lượng ngữ cảnh").
+ *
+ * 1. Tag bump: for every entry p of realloc_pages[n_realloc] (device, may be
+ *    NULL when n_realloc == 0), page_tags[p] += 1 (mod 2^32), once per
+ *    occurrence.  Ids outside [0, P) are skipped.
+ * 2. For token t < T with slot = slot_mapping[t] (device, [T]) in [0, P*ps)
+ *    and every KV head h: FP8 caches store code = E4M3(fl32(x) / s) for each
+ *    element x of k_new[t][h][:] (and v_new[t][h][:]), with IEEE division
+ *    and saturating round-to-nearest-even; in TOKEN mode s = fl32(amax(row)
+ *    / 448) (1 if amax is 0) is computed first and stored at
+ *    scale[page][h][offset].  BF16 caches store the values unchanged.
+ *    Slots < 0 (padding) or >= P*ps are skipped.  Two tokens with the same
+ *    slot in one call race (unspecified result).
+ * k_new: bf16 [T][Hkv][Dk]; v_new: bf16 [T][Hkv][Dv], ignored (may be NULL)
+ * when cache->v_pages is NULL.
+ */
+kvq_status kvq_append(const kvq_cache* cache, const void* k_new, const void* v_new,
+                      const int32_t* slot_mapping, int32_t T, const int32_t* realloc_pages,
+                      int32_t n_realloc, void* stream);
+
+/*
+ * Batched tag validation, a separate launch before decode reads the cache
+ * rather than a check fused into the attention kernel ([remio] "Sicherheit
+ * gemeinsamer KV-Caches wird zum Produktionsthema"; [aifeed] "Kvalita
+ * odpovedí a integrita spoločnej cache"; [lens] "KV キャッシュ整合性チェック").
+ *
+ * For each request b < B: n = clamp(seq_lens[b], 0, max_pages*page_size),
+ * abort_mask[b] = 1 if some i < ceil(n / page_size) has
+ *   block_table[b][i] outside [0, num_pages) or
+ *   page_tags[block_table[b][i]] != expected_tags[b][i],
+ * else 0.  Entries of block_table / expected_tags beyond ceil(n/ps) are not
+ * read.  block_table: i32 [B][max_pages]; expected_tags: u32 [B][max_pages];
+ * seq_lens: i32 [B]; abort_mask: u8 [B] (written).
+ */
+kvq_status kvq_validate(const uint32_t* page_tags, int32_t num_pages, const int32_t* block_table,
+                        const uint32_t* expected_tags, const int32_t* seq_lens,
+                        int32_t page_size, int32_t B, int32_t max_pages, uint8_t* abort_mask,
+                        void* stream);
+
+/*
+ * Bytes of device workspace kvq_decode / kvq_decode_bf16 need for this
+ * cache, batch size and query-head count, with num_ctas persistent blocks
+ * (0 = the library's default for the current device).  Returns 0 for
+ * invalid or unsupported arguments.
+ */
+size_t kvq_decode_workspace_size(const kvq_cache* cache, int32_t B, int32_t num_q_heads,
+                                 int32_t num_ctas);
+
+/*
+ * Decode attention over the paged FP8 cache: each sequence's single new
+ * query token attends to its cached tokens through its page table, with the
+ * E4M3 codes converted to 16-bit values in registers on the way
+ * ([manulx] "Bộ nhớ đệm KV FP8 tăng gấp đôi dung lượng ngữ cảnh"; [remio]
+ * "Warum kleinere Cloudflare-Caches reine Geschwindigkeit schlagen").
+ *
+ *   q           bf16 [B][num_q_heads][Dk]; query head h reads KV head
+ *               h / (num_q_heads / Hkv)
+ *   block_table i32 [B][max_pages]; seq_lens i32 [B] (tokens, clamped to
+ *               [0, max_pages*ps])
+ *   abort_mask  u8 [B] from kvq_validate, or NULL when the check is disabled
+ *               for this deployment; aborted rows read no cache bytes
+ *   out         f32 [B][num_q_heads][Dv]:  sum_j softmax(s)_j * Vhat_j with
+ *               s_j = sm_scale * (q . Khat_j)
+ *   lse         f32 [B][num_q_heads] natural-log sum-exp of s, or NULL
+ *   Aborted or empty rows: out = 0, lse = -inf.
+ *   workspace   device, >= kvq_decode_workspace_size(...) bytes, 256-byte
+ *               aligned; contents on entry are ignored.
+ *   num_ctas    persistent blocks (0 = default); the work is split evenly
+ *               over them regardless of sequence lengths (split-KV), and the
+ *               partial results are merged by a log-sum-exp combine launch.
+ * Page ids outside [0, P) read as zeros (no fault); run kvq_validate first
+ * to abort such requests instead.  Queries must lie within the FP16 range.
+ * Requires cache->dtype == KVQ_FP8_E4M3.  Supported shapes: Dk == Dv in
+ * {64, 128} with separate V pages, ps a multiple of 16 and
+ * num_q_heads / Hkv <= 16; or Dk = 576, Dv = 512 with V aliasing K, one KV
+ * head, 128 query heads, TOKEN scales and ps a multiple of 64.
+ */
+kvq_status kvq_decode(const kvq_cache* cache, const void* q, int32_t num_q_heads,
+                      const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
+                      int32_t B, const uint8_t* abort_mask, float sm_scale, float* out,
+                      float* lse, void* workspace, size_t workspace_bytes, int32_t num_ctas,
+                      void* stream);
+
+/* The same decode over a BF16 cache (cache->dtype == KVQ_BF16), the format
+ * the FP8 cache is compared with ([remio] "Warum kleinere Cloudflare-Caches
+ * reine Geschwindigkeit schlagen").  Same arguments, shapes and rules as
+ * kvq_decode for the Dk == Dv in {64, 128} family. */
+kvq_status kvq_decode_bf16(const kvq_cache* cache, const void* q, int32_t num_q_heads,
+                           const int32_t* block_table, int32_t max_pages,
+                           const int32_t* seq_lens, int32_t B, const uint8_t* abort_mask,
+                           float sm_scale, float* out, float* lse, void* workspace,
+                           size_t workspace_bytes, int32_t num_ctas, void* stream);
+
+/*
+ * Device E4M3 conversion used by kvq_append, exposed for exhaustive checks:
+ * out[i] = E4M3(float with bit pattern start + i), i < count (bit patterns
+ * wrap mod 2^32).  out: u8 [count].
+ */
+kvq_status kvq_e4m3_encode_bits(uint32_t start, uint32_t count, uint8_t* out, void* stream);
+
+/*
+ * Reads and clears the library's device-side error word on the current
+ * device (synchronous).  Bit 0: a pipeline wait in a decode kernel gave up
+ * after its time limit (about one second) and the kernel returned early, so
+ * that launch's outputs are invalid.  *flags_host receives the word.
+ */
+kvq_status kvq_device_error(uint32_t* flags_host);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

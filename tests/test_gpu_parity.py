@@ -1,0 +1,279 @@
+"""GPU parity: libkvq (through its C ABI) against the CPU oracle on the same
+seeded inputs.
+
+Bar: E4M3 codes, page writes, scales, tags and abort masks bit-exact; decode
+outputs within max-abs 2e-3 and max-rel 1e-2 (relative error taken over
+elements with |ref| >= 0.2, where it is meaningful), lse within 2e-3,
+aborted/empty rows exactly 0 / -inf.  Both sides start from the same
+dequantised values; the GPU's error comes from f16 probabilities and FP32
+accumulation order.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fp8_kv_paged_kvq_b200 as kvq
+from fp8_kv_paged_kvq_b200 import workloads as W
+from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch
+from tests import oracle_side as OS
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL, REL_FLOOR = 2e-3, 1e-2, 0.2
+
+
+def assert_decode_close(out, lse, ref_out, ref_lse, what=""):
+    out = out.detach().cpu().double().numpy().reshape(ref_out.shape)
+    lse = lse.detach().cpu().double().numpy().reshape(ref_lse.shape)
+    inf_ref = np.isneginf(ref_lse)
+    assert np.array_equal(np.isneginf(lse), inf_ref), what
+    assert np.all(out[inf_ref] == 0.0), what
+    fin = ~inf_ref
+    d = np.abs(out - ref_out)
+    assert d.max(initial=0.0) <= ATOL, (what, d.max())
+    big = np.abs(ref_out) >= REL_FLOOR
+    if big.any():
+        rel = (d[big] / np.abs(ref_out[big])).max()
+        assert rel <= RTOL, (what, rel)
+    if fin.any():
+        assert np.abs(lse[fin] - ref_lse[fin]).max() <= ATOL, what
+
+
+SPECS = {
+    "tiny": W.spec_by_name("tiny"),
+    "g8_d128_head": W.Spec("g8_d128_head", [1, 15, 16, 17, 300, 1000], 16, 16, 2, 128, 128,
+                           outlier_p=0.01, n_stale=2),
+    "g16_d128": W.Spec("g16_d128", [50, 129, 700], 16, 32, 2, 128, 128),
+    "g3_d64_ps48": W.Spec("g3_d64_ps48", [5, 48, 49, 500], 48, 6, 2, 64, 64,
+                          scale_mode=W.SCALE_TENSOR),
+    "g8_token_ps32": W.Spec("g8_token_ps32", [31, 32, 33, 400], 32, 8, 1, 128, 128,
+                            scale_mode=W.SCALE_TOKEN),
+    "bf16_g8_d128": W.Spec("bf16_g8_d128", [1, 15, 16, 17, 300, 1000], 16, 16, 2, 128, 128,
+                           kv_dtype=W.BF16),
+    "bf16_g12_d64": W.Spec("bf16_g12_d64", [7, 64, 333], 32, 24, 2, 64, 64, kv_dtype=W.BF16),
+    "bf16_g16_d128": W.Spec("bf16_g16_d128", [100, 257], 16, 16, 1, 128, 128, kv_dtype=W.BF16),
+}
+
+
+def build_both(spec, seed=0, num_ctas=0, canary=True):
+    wl = W.make_workload(spec, seed=seed, device="cuda")
+    db = DecodeBatch(wl, num_ctas=num_ctas)
+    if canary and db.cache.fp8:
+        db.cache.k_pages.fill_(0xCD)
+        if db.cache.v_pages is not None:
+            db.cache.v_pages.fill_(0xCD)
+    db.prefill()
+    db.append_new()          # the oracle side's fill() also appends the step's token
+    oc = OS.new_cache(wl)
+    OS.fill(wl, oc)
+    return wl, db, oc
+
+
+@pytest.mark.parametrize("name", list(SPECS))
+def test_append_and_scales_bit_exact(name):
+    wl, db, oc = build_both(SPECS[name], seed=1)
+    db.append_new()
+    torch.cuda.synchronize()
+    c = db.cache
+    if c.fp8:
+        assert np.array_equal(c.k_pages.cpu().numpy(), oc.k_pages)
+        if oc.v_pages is not None:
+            assert np.array_equal(c.v_pages.cpu().numpy(), oc.v_pages)
+        assert np.array_equal(c.k_scale.cpu().numpy(), oc.k_scale)
+        if oc.v_scale is not None:
+            assert np.array_equal(c.v_scale.cpu().numpy(), oc.v_scale)
+    else:
+        assert np.array_equal(c.k_pages.cpu().view(torch.int16).numpy().view(np.uint16), oc.k_pages)
+        assert np.array_equal(c.v_pages.cpu().view(torch.int16).numpy().view(np.uint16), oc.v_pages)
+    assert np.array_equal(c.page_tags.cpu().numpy().view(np.uint32), oc.page_tags)
+
+
+@pytest.mark.parametrize("name", list(SPECS))
+def test_decode_matches_oracle(name):
+    wl, db, oc = build_both(SPECS[name], seed=2)
+    out, lse = db.step(check_tags=True)
+    torch.cuda.synchronize()
+    mask = db.abort.cpu().numpy()
+    ref_mask = oracle.validate(oc.page_tags, wl.block_table, wl.expected_tags, wl.seq_lens,
+                               wl.spec.page_size)
+    assert np.array_equal(mask, ref_mask)
+    want = np.zeros(wl.B, np.uint8)
+    for b, _ in wl.stale:
+        want[b] = 1
+    assert np.array_equal(mask, want)
+    ro, rl = OS.decode(wl, oc, abort=ref_mask)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), name)
+    # with the check disabled every row is decoded
+    out2, lse2 = db.decode(use_abort=False)
+    ro2, rl2 = OS.decode(wl, oc, abort=None)
+    assert_decode_close(out2, lse2, ro2.reshape(out.shape), rl2.reshape(lse.shape), name)
+    assert kvq.device_error() == 0
+
+
+@pytest.mark.parametrize("num_ctas", [1, 2, 3, 7, 64, 148, 296, 1000, 5000])
+def test_split_count_sweep(num_ctas):
+    spec = SPECS["g8_d128_head"]
+    wl, db, oc = build_both(spec, seed=3, num_ctas=num_ctas)
+    out, lse = db.step(check_tags=False)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), str(num_ctas))
+    assert kvq.device_error() == 0
+
+
+def test_page_permutation_is_bit_exact():
+    spec = SPECS["g8_d128_head"]
+    wl, db, _ = build_both(spec, seed=4, canary=False)
+    out1, lse1 = [t.clone() for t in db.step(check_tags=False)]
+    perm = torch.randperm(wl.num_pages, generator=torch.Generator().manual_seed(9)).cuda()
+    c = db.cache
+    k2 = torch.empty_like(c.k_pages)
+    v2 = torch.empty_like(c.v_pages)
+    k2[perm] = c.k_pages
+    v2[perm] = c.v_pages
+    c.k_pages.copy_(k2)
+    c.v_pages.copy_(v2)
+    bt = db.block_table
+    db.block_table = torch.where(bt >= 0, perm[bt.clamp(min=0).long()].int(), bt).contiguous()
+    out2, lse2 = db.decode(use_abort=False)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
+
+
+def test_single_token_returns_value_bit_exact():
+    spec = W.Spec("one", [1, 1, 1], 16, 8, 1, 128, 128)
+    wl, db, oc = build_both(spec, seed=5)
+    out, lse = db.step(check_tags=False)
+    torch.cuda.synchronize()
+    ro, _ = OS.decode(wl, oc)
+    # p = 1: out is exactly fl32(decode(code) * s_v)
+    assert np.array_equal(out.cpu().numpy().reshape(ro.shape), ro.astype(np.float32))
+
+
+def test_aborted_rows_read_nothing():
+    spec = SPECS["g8_d128_head"]
+    wl, db, oc = build_both(spec, seed=6)
+    db.abort.copy_(torch.tensor([1, 0, 1, 0, 0, 1], dtype=torch.uint8))
+    out, lse = db.decode(use_abort=True)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc, abort=np.array([1, 0, 1, 0, 0, 1], np.uint8))
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape))
+    assert torch.all(out[[0, 2, 5]] == 0) and torch.all(torch.isneginf(lse[[0, 2, 5]]))
+
+
+def test_all_rows_aborted_or_empty():
+    spec = W.Spec("empty", [0, 20, 0], 16, 8, 1, 128, 128)
+    wl, db, oc = build_both(spec, seed=7)
+    db.abort.copy_(torch.tensor([0, 1, 0], dtype=torch.uint8))
+    out, lse = db.decode(use_abort=True)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_out_of_range_pages_read_zero_and_validate_aborts():
+    spec = SPECS["g8_d128_head"]
+    wl, db, oc = build_both(spec, seed=8)
+    bt = wl.block_table.copy()
+    bt[4, 3] = wl.num_pages + 5
+    bt[5, 0] = -7
+    wl.block_table = bt
+    db.block_table = torch.from_numpy(bt).cuda()
+    m = db.validate()
+    ref = oracle.validate(oc.page_tags, bt, wl.expected_tags, wl.seq_lens, spec.page_size)
+    torch.cuda.synchronize()
+    assert np.array_equal(m.cpu().numpy(), ref) and ref[4] == 1 and ref[5] == 1
+    out, lse = db.decode(use_abort=False)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape))
+
+
+def test_validate_random_bit_exact():
+    r = np.random.default_rng(0)
+    for trial in range(30):
+        P, B, maxp, ps = int(r.integers(1, 3000)), int(r.integers(1, 40)), int(r.integers(1, 5000)), int(r.integers(1, 33))
+        tags = r.integers(0, 3, P).astype(np.uint32)
+        bt = r.integers(-2, P + 2, (B, maxp)).astype(np.int32)
+        bt[r.random((B, maxp)) < 0.999] = r.integers(0, P, 1)[0]
+        exp = tags[np.clip(bt, 0, P - 1)].copy()
+        flip = r.random((B, maxp)) < 2e-4
+        exp[flip] ^= 1
+        lens = r.integers(-3, maxp * ps + 5, B).astype(np.int32)
+        got = kvq.validate(torch.from_numpy(tags.view(np.int32)).cuda(), torch.from_numpy(bt).cuda(),
+                           torch.from_numpy(exp.view(np.int32)).cuda(), torch.from_numpy(lens).cuda(), ps)
+        ref = oracle.validate(tags, bt, exp, lens, ps)
+        assert np.array_equal(got.cpu().numpy(), ref), trial
+
+
+def test_tag_bump_matches_oracle():
+    P = 50
+    tags = np.random.default_rng(1).integers(0, 2**32, P, dtype=np.uint64).astype(np.uint32)
+    tags[3] = 0xFFFFFFFF
+    realloc = np.array([3, 3, 7, -1, 50, 49, 0, 7, 7], np.int32)
+    c = kvq.PagedCache(kvq.FP8_E4M3, kvq.SCALE_HEAD, P, 16, 1, 16, 16,
+                       tags=torch.from_numpy(tags.view(np.int32)))
+    kvq.append(c, torch.zeros((0, 1, 16), dtype=torch.bfloat16, device="cuda"),
+               torch.zeros((0, 1, 16), dtype=torch.bfloat16, device="cuda"),
+               torch.zeros(0, dtype=torch.int32, device="cuda"),
+               realloc_pages=torch.from_numpy(realloc).cuda())
+    oc = oracle.Cache(oracle.FP8, oracle.SCALE_HEAD, P, 16, 1, 16, 16,
+                      np.zeros((P, 1, 16, 16), np.uint8), np.zeros((P, 1, 16, 16), np.uint8),
+                      np.ones(1, np.float32), np.ones(1, np.float32), tags.copy())
+    oracle.append(oc, np.zeros((0, 1, 16), np.uint16), np.zeros((0, 1, 16), np.uint16),
+                  np.zeros(0, np.int32), realloc_pages=realloc)
+    assert np.array_equal(c.page_tags.cpu().numpy().view(np.uint32), oc.page_tags)
+
+
+def test_amax_chunked_and_nan():
+    x = torch.randn(1000, 3, 64, device="cuda").to(torch.bfloat16)
+    x[5, 1, 7] = float("nan")
+    a = torch.zeros(3, device="cuda")
+    for lo in range(0, 1000, 300):
+        kvq.amax(x[lo:lo + 300].contiguous(), True, a)
+    s = kvq.scale_from_amax(a)
+    torch.cuda.synchronize()
+    want = oracle.scales(OS.bf16_bits(x), per_head=True)
+    assert np.array_equal(s.cpu().numpy(), want)
+    s1 = kvq.scale_from_amax(kvq.amax(x, False))
+    assert np.array_equal(s1.cpu().numpy(), oracle.scales(OS.bf16_bits(x), per_head=False))
+
+
+def test_e4m3_encode_all_2_32_patterns():
+    """Device conversion vs the oracle's integer-arithmetic encoder, every float bit pattern."""
+    chunk = 1 << 28
+    dev = torch.empty(chunk, dtype=torch.uint8, device="cuda")
+    for i in range((1 << 32) // chunk):
+        start = i * chunk
+        kvq.e4m3_encode_bits(start, chunk, dev)
+        ref = oracle.e4m3_encode_bits_range(start, chunk)
+        got = dev.cpu().numpy()
+        if not np.array_equal(got, ref):
+            bad = np.nonzero(got != ref)[0][:5]
+            raise AssertionError([(hex(start + int(j)), hex(got[j]), hex(ref[j])) for j in bad])
+
+
+def test_host_argument_errors():
+    c = kvq.PagedCache(kvq.FP8_E4M3, kvq.SCALE_HEAD, 4, 16, 1, 128, 128)
+    q = torch.zeros((1, 8, 128), dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros((1, 1), dtype=torch.int32, device="cuda")
+    sl = torch.ones(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.decode(c, q, bt, sl, None, 1.0, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == kvq.KVQ_ERR_WORKSPACE
+    q7 = torch.zeros((1, 7, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(kvq.KvqError):
+        kvq.decode(c, q7, bt, sl, None, 1.0, workspace=torch.empty(1 << 20, dtype=torch.uint8, device="cuda"))
+    cb = kvq.PagedCache(kvq.BF16, kvq.SCALE_HEAD, 4, 16, 1, 128, 128)
+    ws = kvq.alloc_workspace(cb, 1, 8)
+    with pytest.raises(kvq.KvqError) as e:   # fp8 entry point on a bf16 cache
+        kvq.lib().kvq_decode  # noqa: B018
+        import ctypes
+        st = kvq.lib().kvq_decode(ctypes.byref(cb.desc), ctypes.c_void_p(q.data_ptr()), 8,
+                                  ctypes.c_void_p(bt.data_ptr()), 1, ctypes.c_void_p(sl.data_ptr()),
+                                  1, None, ctypes.c_float(1.0), ctypes.c_void_p(q.data_ptr()), None,
+                                  ctypes.c_void_p(ws.data_ptr()), ws.numel(), 0, None)
+        kvq._check("kvq_decode", st)
+    assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
