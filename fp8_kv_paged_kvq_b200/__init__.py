@@ -10,6 +10,7 @@ Entry points mirror include/kvq.h:
     append                   tag bump on reallocation + quantize-on-append
     validate                 batched page-tag check -> abort mask
     decode, decode_bf16      split-KV paged decode attention (+ LSE combine)
+    decode_noalloc           FP8 decode using the library's fixed scratch array
     e4m3_encode_bits         the device E4M3 conversion, for exhaustive checks
     device_error             read/clear the device-side error word
 """
@@ -71,10 +72,13 @@ def lib() -> ctypes.CDLL:
                _VP, _VP, _VP, ctypes.c_size_t, _I32, _VP]
         L.kvq_decode.argtypes = dec
         L.kvq_decode_bf16.argtypes = dec
+        L.kvq_decode_noalloc.argtypes = [ctypes.POINTER(KvqCacheDesc), _VP, _I32, _VP, _I32, _VP,
+                                         _I32, _VP, ctypes.c_float, _VP, _VP, _I32, _VP]
         L.kvq_e4m3_encode_bits.argtypes = [_U32, _U32, _VP, _VP]
         L.kvq_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
         for f in ("kvq_amax", "kvq_scale_from_amax", "kvq_append", "kvq_validate", "kvq_decode",
-                  "kvq_decode_bf16", "kvq_e4m3_encode_bits", "kvq_device_error"):
+                  "kvq_decode_bf16", "kvq_decode_noalloc", "kvq_e4m3_encode_bits",
+                  "kvq_device_error"):
             getattr(L, f).restype = _I32
         _lib = L
     return _lib
@@ -229,6 +233,21 @@ def decode(cache: PagedCache, q: torch.Tensor, block_table: torch.Tensor, seq_le
 
 
 decode_bf16 = decode
+
+
+def decode_noalloc(cache: PagedCache, q: torch.Tensor, block_table: torch.Tensor,
+                   seq_lens: torch.Tensor, abort_mask: Optional[torch.Tensor], sm_scale: float,
+                   out: torch.Tensor, lse: Optional[torch.Tensor], num_ctas: int = 0, stream=None):
+    """FP8 decode whose scratch is the library's fixed device array (no workspace argument).
+
+    For callers that cannot allocate device memory; out / lse must be given.  Calls on one
+    device share the array, so order them on one stream."""
+    B, Hq, _ = q.shape
+    _check("kvq_decode_noalloc", lib().kvq_decode_noalloc(
+        ctypes.byref(cache.desc), _ptr(q), Hq, _ptr(block_table), block_table.shape[1],
+        _ptr(seq_lens), B, _ptr(abort_mask), ctypes.c_float(sm_scale), _ptr(out), _ptr(lse),
+        num_ctas, _stream(stream)))
+    return out, lse
 
 
 def e4m3_encode_bits(start: int, count: int, out: Optional[torch.Tensor] = None, stream=None):

@@ -4,3 +4,4 @@
 #include "validate.cu"
 #include "decode_gqa.cu"
 #include "api.cu"
+#include "decode_noalloc.cu"

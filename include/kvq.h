@@ -213,6 +213,31 @@ kvq_status kvq_decode_bf16(const kvq_cache* cache, const void* q, int32_t num_q_
                            size_t workspace_bytes, int32_t num_ctas, void* stream);
 
 /*
+ * kvq_decode without a caller-provided workspace.  The source pages have no
+ * counterpart to this call: it exists for callers that cannot allocate
+ * device memory, such as a plug-in inside a host framework that owns all
+ * device memory and hands out none, or a serving loop that forbids any
+ * allocation after start-up.  Same arguments, rules and results as
+ * kvq_decode (FP8 caches only) minus `workspace` / `workspace_bytes`.
+ *
+ * The scratch lives in a fixed 8 MiB array inside libkvq.so that every GPU
+ * which loads the library holds until the process exits.  A batch whose
+ * workspace (kvq_decode_workspace_size) exceeds 8 MiB is rejected with
+ * KVQ_ERR_WORKSPACE before anything is enqueued; the allocating kvq_decode
+ * has no such limit.  The call allocates nothing.  The first call on each
+ * device looks up the array's device address (with that device current);
+ * make that first call before any stream capture.  All calls on a device
+ * share the array, so calls that overlap on the GPU (e.g. on two unordered
+ * streams) race and give undefined results; order them on one stream.
+ * Nothing in the array needs to start at zero.
+ */
+kvq_status kvq_decode_noalloc(const kvq_cache* cache, const void* q, int32_t num_q_heads,
+                              const int32_t* block_table, int32_t max_pages,
+                              const int32_t* seq_lens, int32_t B, const uint8_t* abort_mask,
+                              float sm_scale, float* out, float* lse, int32_t num_ctas,
+                              void* stream);
+
+/*
  * Device E4M3 conversion used by kvq_append, exposed for exhaustive checks:
  * out[i] = E4M3(float with bit pattern start + i), i < count (bit patterns
  * wrap mod 2^32).  out: u8 [count].
