@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--loop-steps", type=int, default=1000,
+                    help="decode steps of the long workload's loop")
     ap.add_argument("--seqs", type=int, default=0,
                     help="keep only the first N sequences (smaller case for profiling)")
     return ap.parse_args()
@@ -428,6 +430,104 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_long(args):
+    """The long workload as its decode loop: every step appends one token per
+    sequence with page reallocation and tag bumps; even steps validate with
+    0.01% of expected tags made stale (those requests abort for that step), odd
+    steps skip the check.  Step time = device time of append + validate +
+    decode replayed from a CUDA graph; bytes count decoded (non-aborted) rows."""
+    rank, world, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import fp8_kv_paged_kvq_b200 as kvq
+    from fp8_kv_paged_kvq_b200 import build as kvq_build
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    from fp8_kv_paged_kvq_b200.pipeline import DecodeLoop
+    if rank == 0:
+        kvq_build.build()
+    barrier(world)
+    spec = W.spec_by_name("long")
+    wl = W.make_workload(spec, seed=0, device=dev)
+    steps = args.loop_steps
+    loop = DecodeLoop(wl, steps, device=dev, num_ctas=args.num_ctas)
+    loop.batch.prefill()
+    torch.cuda.synchronize()
+    row = spec.num_kv_heads * (spec.head_dim_k + spec.head_dim_v)
+    stream = torch.cuda.Stream(device=dev)
+    recs = []
+    with torch.cuda.stream(stream):
+        loop.capture(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        sampler = ClockSampler(local)
+        with sampler:
+            for ls in W.loop_steps(wl, steps):
+                kind = ls.step % 3          # 0: check + stale tags, 1: clean check, 2: no check
+                chk = kind != 2
+                idx = loop.prepare(ls, chk, inject_stale=(kind == 0))
+                ev = loop.run(chk, stream)
+                loop.restore(idx)
+                torch.cuda.synchronize()
+                t_app, t_val, t_dec = (ev[i].elapsed_time(ev[i + 1]) for i in range(3))
+                aborted = {b for b, _ in ls.stale} if kind == 0 else set()
+                kv = sum(int(ls.seq_lens[b]) for b in range(spec.B) if b not in aborted) * row
+                recs.append((kind, t_app, t_val, t_dec, kv, len(aborted)))
+    assert kvq.device_error() == 0, "device-side wait timed out"
+    kind = np.array([r[0] for r in recs])
+    t_app = np.array([r[1] for r in recs])
+    t_val = np.array([r[2] for r in recs])
+    t_dec = np.array([r[3] for r in recs])
+    kv = np.array([r[4] for r in recs], dtype=np.float64)
+    ms = t_app + t_val + t_dec
+    # the tracker's view must match what the device did
+    host_tags = loop.tracker.tags
+    dev_tags = loop.batch.cache.page_tags.cpu().numpy().view(np.uint32)
+    tags_ok = bool(np.array_equal(host_tags, dev_tags))
+    def mean(x):
+        return float(max_over_ranks(float(np.mean(x)), world))
+    step_clean, step_nochk = mean(ms[kind == 1]), mean(ms[kind == 2])
+    # the no-check graph records the same events around an empty slot: its gap is
+    # the event overhead, subtracted from the validate slot
+    val = mean(t_val[kind == 1]) - mean(t_val[kind == 2])
+    gbs = world * kv.sum() / (max_over_ranks(float(ms.sum()), world) * 1e-3) / 1e9
+    hbm, hbm_kind = peaks()
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
+        "warmup": 1, "ms_per_step": float(ms.mean()), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 mma / f32 accumulate (e4m3 cache)", "data": "synthetic",
+        "config": {"workload": workload_desc("long"),
+                   "loop": f"{steps} steps: append 1 token/seq with page reallocation + tag "
+                           "bump; steps cycle validate+stale tags / validate / no validation",
+                   "l2": "inputs exceed L2: >3 GB of cache read per step",
+                   "timing": "CUDA graph per step between CUDA events"},
+        "decode_tokens_per_s": world * spec.B / (ms.mean() * 1e-3),
+        "hbm_frac_of_step": gbs / world / hbm,
+        "ms_per_step_with_validation": step_clean,
+        "ms_per_step_without_validation": step_nochk,
+        "ms_per_step_with_validation_and_stale_tags": mean(ms[kind == 0]),
+        "p95_ms_with_validation": float(np.percentile(ms[kind == 1], 95)),
+        "p95_ms_without_validation": float(np.percentile(ms[kind == 2], 95)),
+        "ms_validate_kernel": val,
+        "ms_decode_with_validation": mean(t_dec[kind == 1]),
+        "ms_decode_without_validation": mean(t_dec[kind == 2]),
+        "ms_decode_with_stale_aborts": mean(t_dec[kind == 0]),
+        "ms_append": mean(t_app),
+        "validate_overhead_pct": 100.0 * (step_clean - step_nochk) / step_nochk,
+        "validate_overhead_note": "steps cycle: validate with 0.01% stale tags / validate with "
+                                  "clean tags / no validation; overhead compares the last two",
+        "aborted_requests_per_stale_step": float(np.mean([r[5] for r in recs if r[0] == 0])),
+        "pages_reallocated": int(sum(len(l.new_pages) for l in W.loop_steps(wl, steps))),
+        "host_tracker_matches_device_tags": tags_ok,
+        "clocks": sampler.summary(), "gpu_launches": int(4 * np.sum(kind != 2) + 3 * np.sum(kind == 2)),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def run_e2e(db, args, stream, kv_bytes, world):
     """Same step through the Python API, step inputs copied from pinned host
     memory and the result read back, every step."""
@@ -501,6 +601,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "long":
+        run_long(args)
     else:
         run_ours(args)
 

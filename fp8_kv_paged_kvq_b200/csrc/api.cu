@@ -216,7 +216,6 @@ kvq_status kvq_validate(const uint32_t* page_tags, int32_t num_pages, const int3
   if (page_tags == nullptr || block_table == nullptr || expected_tags == nullptr ||
       seq_lens == nullptr || abort_mask == nullptr)
     return KVQ_ERR_INVALID_ARG;
-  if (B > 65535) return KVQ_ERR_UNSUPPORTED;
   return from_cuda(launch_validate(page_tags, num_pages, block_table, expected_tags, seq_lens,
                                    page_size, B, max_pages, abort_mask,
                                    static_cast<cudaStream_t>(stream)));

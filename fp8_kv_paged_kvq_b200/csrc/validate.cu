@@ -6,58 +6,76 @@
 // modelov Kimi a GLM kompresiou cache a váh" (aifeed.sk), section "Kvalita
 // odpovedí a integrita spoločnej cache".
 //
-// Grid: (chunks of kChunk entries, B).  The mask is cleared by a memset on
-// the same stream first; a block that finds a bad entry writes 1.  The cost
-// is launch latency plus two dependent loads per entry (the block table /
-// expected tag, then the live-tag gather), so each thread keeps kPerThread
-// independent entries in flight.
+// Each request gets a thread-block cluster of C <= 8 CTAs, enough that one
+// round of loads covers its block-table row: CTA r checks entries
+// r*kPerCta + k*kValThreads + tid (+ C*kPerCta per further round).  The CTAs
+// combine their flags through distributed shared memory and rank 0 writes the
+// request's mask byte, so no separate clear is needed.  The cost is launch
+// latency plus, after the sequence length, two dependent loads per entry:
+// the block-table entry with its expected tag, then the live tag.
+#include <cooperative_groups.h>
+
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
+namespace cg = cooperative_groups;
 
-constexpr int kValThreads = 256;
+constexpr int kValThreads = 512;
 constexpr int kPerThread = 8;
-constexpr int kChunk = kValThreads * kPerThread;
+constexpr int kPerCta = kValThreads * kPerThread;
+constexpr int kMaxCluster = 8;
 
 __global__ void __launch_bounds__(kValThreads)
     validate_kernel(const uint32_t* __restrict__ tags, int32_t P,
                     const int32_t* __restrict__ block_table,
                     const uint32_t* __restrict__ expected, const int32_t* __restrict__ seq_lens,
                     int32_t ps, int32_t max_pages, uint8_t* __restrict__ abort_mask) {
-  const int32_t b = blockIdx.y;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int32_t b = blockIdx.x / C;
+  __shared__ int flag;
   int64_t n = seq_lens[b];
   n = n < 0 ? 0 : n;
   const int64_t cap = static_cast<int64_t>(max_pages) * ps;
   n = n > cap ? cap : n;
   const int32_t npages = static_cast<int32_t>((n + ps - 1) / ps);
-  const int32_t base = blockIdx.x * kChunk;
-  if (base >= npages) return;                          // block-uniform
   const int32_t* bt = block_table + static_cast<int64_t>(b) * max_pages;
   const uint32_t* ex = expected + static_cast<int64_t>(b) * max_pages;
-  int32_t page[kPerThread];
-  uint32_t want[kPerThread];
-#pragma unroll
-  for (int k = 0; k < kPerThread; ++k) {
-    const int32_t i = base + k * kValThreads + threadIdx.x;   // coalesced
-    page[k] = 0;
-    want[k] = 0;
-    if (i < npages) {
-      page[k] = bt[i];
-      want[k] = ex[i];
-    }
-  }
   int bad = 0;
+  for (int32_t base = rank * kPerCta; base < npages; base += C * kPerCta) {
+    int32_t page[kPerThread];
+    uint32_t want[kPerThread];
 #pragma unroll
-  for (int k = 0; k < kPerThread; ++k) {
-    const int32_t i = base + k * kValThreads + threadIdx.x;
-    if (i < npages) {
-      const int32_t p = page[k];
-      if (p < 0 || p >= P) bad = 1;
-      else if (tags[p] != want[k]) bad = 1;
+    for (int k = 0; k < kPerThread; ++k) {
+      const int32_t i = base + k * kValThreads + threadIdx.x;   // coalesced
+      page[k] = 0;
+      want[k] = 0;
+      if (i < npages) {
+        page[k] = bt[i];
+        want[k] = ex[i];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int32_t i = base + k * kValThreads + threadIdx.x;
+      if (i < npages) {
+        const int32_t p = page[k];
+        if (p < 0 || p >= P) bad = 1;
+        else if (tags[p] != want[k]) bad = 1;
+      }
     }
   }
-  if (__syncthreads_or(bad) && threadIdx.x == 0) abort_mask[b] = 1;
+  const int any = __syncthreads_or(bad);
+  if (threadIdx.x == 0) flag = any;
+  cluster.sync();
+  if (rank == 0 && threadIdx.x == 0) {
+    int all = 0;
+    for (int r = 0; r < C; ++r) all |= *cluster.map_shared_rank(&flag, r);
+    abort_mask[b] = all ? 1 : 0;
+  }
+  cluster.sync();   // every CTA's flag stays alive until rank 0 has read it
 }
 
 cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* block_table,
@@ -65,12 +83,22 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
                             int32_t B, int32_t max_pages, uint8_t* abort_mask,
                             cudaStream_t stream) {
   if (B == 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(abort_mask, 0, static_cast<size_t>(B), stream);
-  if (e != cudaSuccess) return e;
-  dim3 grid((max_pages + kChunk - 1) / kChunk, B);
-  validate_kernel<<<grid, kValThreads, 0, stream>>>(tags, P, block_table, expected, seq_lens, ps,
-                                                    max_pages, abort_mask);
-  return cudaGetLastError();
+  int C = (max_pages + kPerCta - 1) / kPerCta;
+  C = C < 1 ? 1 : (C > kMaxCluster ? kMaxCluster : C);
+  if (static_cast<int64_t>(B) * C > 0x7fffffff) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(B * C));
+  cfg.blockDim = dim3(kValThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, validate_kernel, tags, P, block_table, expected, seq_lens, ps,
+                            max_pages, abort_mask);
 }
 
 cudaError_t read_and_clear_error_flags(uint32_t* flags) {

@@ -88,3 +88,103 @@ class DecodeBatch:
         if check_tags:
             self.validate(stream)
         return self.decode(use_abort=check_tags, stream=stream)
+
+
+class DecodeLoop:
+    """The long decode loop on the device.  Every step appends one token per
+    sequence (pages handed out from the free list are reallocations whose tags
+    kvq_append bumps), validates the tracker's expected tags with some entries
+    made stale for that step (or skips the check), and decodes.
+
+    The hot path of a step (kvq_append -> kvq_validate -> kvq_decode) is a CUDA
+    graph over fixed device buffers, so its kernels run back to back; the
+    realloc list is padded to B entries with -1 (skipped by kvq_append).
+    Page-table bookkeeping for the step is written into those buffers first."""
+
+    def __init__(self, wl: W.Workload, steps: int, device="cuda", num_ctas: int = 0):
+        from .paging import TagTracker
+        s = wl.spec
+        self.wl, self.steps = wl, steps
+        self.device = torch.device(device)
+        cap = W.loop_capacity(wl, steps)
+        self.cap = cap
+        self.tracker = TagTracker(wl.page_tags, wl.block_table, wl.seq_lens, s.page_size, cap)
+        self.batch = DecodeBatch(wl, device=device, num_ctas=num_ctas)
+        db = self.batch
+        db.block_table = _dev_i32(self.tracker.block_table, self.device)
+        db.expected = _dev_i32(self.tracker.expected, self.device)
+        self.realloc = torch.full((s.B,), -1, dtype=torch.int32, device=self.device)
+        self.graphs = {}
+
+    def _path(self, check_tags: bool, stream=None, ev=None):
+        db = self.batch
+        st = torch.cuda.current_stream() if stream is None else stream
+        if ev is not None:
+            ev[0].record(st)
+        append(db.cache, db.k_new, db.v_new, db.new_slots, self.realloc, stream)
+        if ev is not None:
+            ev[1].record(st)
+        if check_tags:
+            db.validate(stream)
+        if ev is not None:
+            ev[2].record(st)
+        db.decode(use_abort=check_tags, stream=stream)
+        if ev is not None:
+            ev[3].record(st)
+
+    def capture(self, stream) -> None:
+        """Capture the step's hot path, with and without the tag check, with timing
+        events between append, validate and decode recorded inside the graph."""
+        for chk in (True, False):
+            self._path(chk, stream)          # warm up outside capture
+            ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                self._path(chk, stream, ev)
+            self.graphs[chk] = (g, ev)
+
+    def _flat(self, entries):
+        return torch.tensor([b * self.cap + i for b, i in entries], dtype=torch.long,
+                            device=self.device)
+
+    def prepare(self, ls: W.LoopStep, check_tags: bool, inject_stale: bool = True):
+        """Write the step's inputs into the fixed buffers; with check_tags and
+        inject_stale, the step's stale entries are corrupted in the expected tags.
+        Returns the stale-entry index (restore() undoes it after the step)."""
+        db = self.batch
+        pages, tags, entries = [], [], []
+        for b, i, page in ls.new_pages:
+            tags.append(self.tracker.hand_out(b, i, page))
+            pages.append(page)
+            entries.append((b, i))
+        if entries:
+            idx = self._flat(entries)
+            db.block_table.view(-1)[idx] = torch.tensor(pages, dtype=torch.int32,
+                                                        device=self.device)
+            db.expected.view(-1)[idx] = torch.from_numpy(
+                np.array(tags, np.uint32).view(np.int32)).to(self.device)
+        rl = np.full(self.wl.spec.B, -1, np.int32)
+        rl[: len(pages)] = pages
+        self.realloc.copy_(torch.from_numpy(rl))
+        db.seq_lens.copy_(torch.from_numpy(ls.seq_lens))
+        db.new_slots.copy_(torch.from_numpy(ls.slots))
+        k, v = W.loop_tokens(self.wl, ls.step)
+        db.k_new.copy_(k)
+        if v is not None:
+            db.v_new.copy_(v)
+        stale_idx = self._flat(ls.stale) if (check_tags and inject_stale and ls.stale) else None
+        if stale_idx is not None:
+            db.expected.view(-1)[stale_idx] ^= 1
+        return stale_idx
+
+    def restore(self, stale_idx) -> None:
+        if stale_idx is not None:
+            self.batch.expected.view(-1)[stale_idx] ^= 1
+
+    def run(self, check_tags: bool, stream):
+        """Replay the step's graph.  Returns its four events (before append, before
+        validate, before decode, after decode); they are reused by the next replay of
+        the same graph, so read them after synchronizing and before replaying again."""
+        g, ev = self.graphs[check_tags]
+        g.replay()
+        return ev

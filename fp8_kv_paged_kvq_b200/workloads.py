@@ -232,3 +232,69 @@ def make_workload(spec: Spec, seed: int = 0, device="cpu") -> Workload:
     sm = spec.sm_scale if spec.sm_scale is not None else 1.0 / math.sqrt(spec.head_dim_k)
     return Workload(spec, seed, device, P, lens, bt, tags, expected, stale, free, hist_slots,
                     new_slots, float(sm))
+
+
+# ---------------------------------------------------------------------------
+# The multi-step decode loop (long workload): layout of every step
+# ---------------------------------------------------------------------------
+@dataclass
+class LoopStep:
+    step: int
+    slots: np.ndarray            # int32 [B]: slot of each sequence's new token
+    new_pages: List[tuple]       # (b, i, page): entry i of sequence b handed out this step
+    seq_lens: np.ndarray         # int32 [B]: tokens each sequence decodes over this step
+    stale: List[tuple]           # (b, i): expected-tag entries made stale for this step
+
+
+def loop_capacity(wl: Workload, steps: int) -> int:
+    """Block-table width that holds every sequence after `steps` steps."""
+    ps = wl.spec.page_size
+    return int(((wl.seq_lens.astype(np.int64) + steps - 1 + ps - 1) // ps).max())
+
+
+def loop_steps(wl: Workload, steps: int) -> Iterator[LoopStep]:
+    """Step s appends token seq_len-1+s of every sequence (step 0 appends the
+    workload's own new token) and decodes over seq_len+s tokens.  A token that
+    starts a page takes the next page of the seeded free list.  Each step
+    re-draws ceil(stale_frac * entries) stale (request, entry) positions."""
+    s = wl.spec
+    ps = s.page_size
+    free = list(wl.free_pages.tolist())
+    npages = ((wl.seq_lens.astype(np.int64) + ps - 1) // ps).astype(np.int64)
+    bt = {b: list(wl.block_table[b, : npages[b]]) for b in range(s.B)}
+    for st in range(steps):
+        pos = wl.seq_lens.astype(np.int64) - 1 + st
+        slots = np.full(s.B, -1, np.int32)
+        new_pages = []
+        for b in range(s.B):
+            if wl.seq_lens[b] == 0:
+                continue
+            i = int(pos[b] // ps)
+            if i >= len(bt[b]):
+                page = free.pop(0)
+                bt[b].append(page)
+                new_pages.append((b, i, page))
+            slots[b] = bt[b][i] * ps + pos[b] % ps
+        lens = np.where(wl.seq_lens > 0, wl.seq_lens + st, 0).astype(np.int32)
+        stale = []
+        if s.stale_frac:
+            ent = ((lens.astype(np.int64) + ps - 1) // ps)
+            n = int(math.ceil(s.stale_frac * ent.sum()))
+            r = _rng(wl.seed, s.name, "stale", st)
+            flat = r.choice(int(ent.sum()), size=n, replace=False)
+            starts = np.concatenate([[0], np.cumsum(ent)])
+            for f in sorted(flat.tolist()):
+                b = int(np.searchsorted(starts, f, side="right") - 1)
+                stale.append((b, int(f - starts[b])))
+        yield LoopStep(st, slots, new_pages, lens, stale)
+
+
+def loop_tokens(wl: Workload, step: int):
+    """Random K/V of the token each sequence appends at `step` (step 0: the workload's own)."""
+    if step == 0:
+        k, v, _ = wl.new_tokens()
+        return k, v
+    s = wl.spec
+    k = wl._normal((s.B, s.num_kv_heads, s.head_dim_k), "loopk", step)
+    v = None if s.v_alias else wl._normal((s.B, s.num_kv_heads, s.head_dim_v), "loopv", step)
+    return k, v

@@ -94,6 +94,16 @@ def scales(x_bf16_bits: np.ndarray, per_head: bool) -> np.ndarray:
     return out
 
 
+def amax(x_bf16_bits: np.ndarray, per_head: bool, out: np.ndarray) -> np.ndarray:
+    """Fold max|x| of a BF16 tensor [T][H][D] into out ([1] or [H] float32), in place."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    T, H, D = x.shape
+    assert out.dtype == np.float32 and out.flags["C_CONTIGUOUS"]
+    lib().oracle_amax(_p(x), ctypes.c_int64(T), ctypes.c_int32(H), ctypes.c_int32(D),
+                      ctypes.c_int32(1 if per_head else 0), _p(out))
+    return out
+
+
 class Cache:
     """Host copy of a paged cache: the same fields the CUDA library's cache descriptor holds."""
 

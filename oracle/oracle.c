@@ -147,23 +147,29 @@ float oracle_scale_from_amax(float amax) {
   return amax / 448.0f;   /* IEEE binary32 division, correctly rounded */
 }
 
+/* Fold max|x| of a BF16 tensor x[T][H][D] into amax_io[1] (per_head == 0)
+ * or amax_io[H] (per_head != 0); NaN elements are ignored (v > amax is
+ * false for them). */
+void oracle_amax(const uint16_t* x, int64_t T, int32_t H, int32_t D, int32_t per_head,
+                 float* amax_io) {
+  for (int64_t t = 0; t < T; t++)
+    for (int32_t h = 0; h < H; h++) {
+      float* a = amax_io + (per_head ? h : 0);
+      for (int32_t d = 0; d < D; d++) {
+        float v = fabsf(oracle_bf16_to_f32(x[(t * H + h) * D + d]));
+        if (v > *a) *a = v;
+      }
+    }
+}
+
 /* Scales of a BF16 tensor x[T][H][D]: one over everything (per_head == 0)
  * or one per head (per_head != 0). */
 void oracle_scales(const uint16_t* x, int64_t T, int32_t H, int32_t D, int32_t per_head,
                    float* scale_out) {
   int32_t nout = per_head ? H : 1;
-  for (int32_t o = 0; o < nout; o++) {
-    float amax = 0.0f;
-    for (int64_t t = 0; t < T; t++)
-      for (int32_t h = 0; h < H; h++) {
-        if (per_head && h != o) continue;
-        for (int32_t d = 0; d < D; d++) {
-          float v = fabsf(oracle_bf16_to_f32(x[(t * H + h) * D + d]));
-          if (v > amax) amax = v;
-        }
-      }
-    scale_out[o] = oracle_scale_from_amax(amax);
-  }
+  for (int32_t o = 0; o < nout; o++) scale_out[o] = 0.0f;
+  oracle_amax(x, T, H, D, per_head, scale_out);
+  for (int32_t o = 0; o < nout; o++) scale_out[o] = oracle_scale_from_amax(scale_out[o]);
 }
 
 /* ------------------------------------------------------------------ */
@@ -192,6 +198,8 @@ void oracle_append(int32_t dtype, int32_t scale_mode, int32_t P, int32_t ps, int
     int32_t p = realloc_pages[r];
     if (p >= 0 && p < P) tags[p] = tags[p] + 1u;
   }
+  /* tokens write disjoint rows (distinct slots), so they are independent */
+#pragma omp parallel for schedule(static)
   for (int32_t t = 0; t < T; t++) {
     int64_t slot = slot_mapping[t];
     if (slot < 0 || slot >= (int64_t)P * ps) continue;
