@@ -36,6 +36,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "FP8 paged decode attention: KV GB/s (% of HBM peak) and decode tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse():
@@ -82,6 +83,45 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 TFLOP/s of this GPU (burst: the decode launch is timed on its own)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def is_wide(spec) -> bool:
+    """The 128-query-head, one-KV-head shape served by the tensor-core kernel."""
+    return spec.num_q_heads // spec.num_kv_heads >= 64
+
+
+def decode_roofline(spec, wl, alg_bytes, ms_dec, traffic):
+    """Roofline of one kvq_decode launch.  The 8-head kernel moves bytes
+    (bound: HBM).  The wide kernel is a pair of dense contractions per token,
+    QK^T (a bf16 query against keys that are exact in f16) and PV (f16), so it
+    is bound by the tensor cores at the f16/bf16 rate: 2 * Hq * (Dk + Dv) FLOPs
+    per decoded token."""
+    if is_wide(spec):
+        tokens = int(np.minimum(wl.seq_lens, wl.max_pages * spec.page_size).sum())
+        flops = 2.0 * spec.num_q_heads * (spec.head_dim_k + spec.head_dim_v) * tokens
+        peak, kind = tensor_peak()
+        achieved = flops / (ms_dec * 1e-3) / 1e12
+        return {"bound": "tensor",
+                "kernel": "kvq_decode (wide_prep_kernel + wide_decode_kernel + lse_combine_kernel)",
+                "achieved": achieved, "peak": peak, "peak_kind": kind + " (bf16 burst)",
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
+                "ms_per_launch": ms_dec}
+    hbm, kind = peaks()
+    achieved = alg_bytes / (ms_dec * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "kvq_decode (gqa_decode_kernel + lse_combine_kernel)",
+            "achieved": achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": traffic,
+            "algorithmic_bytes_per_launch": alg_bytes, "ms_per_launch": ms_dec}
 
 
 # ---------------------------------------------------------------------------
@@ -395,7 +435,9 @@ def run_ours(args):
         bf16 = run_bf16(wl, args, stream, world, dev)
 
     value = world * kv_bytes / (ms_step * 1e-3) / 1e9
-    achieved = alg_bytes / (ms_dec * 1e-3) / 1e9
+    # kernels per step: append, validate, then decode (wide: query pre-pass +
+    # decode + combine; otherwise decode + combine)
+    launches = 2 + (3 if is_wide(s) else 2)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -410,11 +452,9 @@ def run_ours(args):
         "hbm_frac_of_step": value / world / hbm,
         "validate_overhead_pct": 100.0 * (ms_step - ms_nochk) / ms_nochk,
         "ms_per_step_without_validation": ms_nochk,
-        "roofline": {"bound": "hbm", "kernel": "kvq_decode (gqa_decode_kernel + lse_combine_kernel)",
-                     "achieved": achieved, "peak": hbm, "peak_kind": hbm_kind, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": measured_traffic(args.workload, args.seqs),
-                     "algorithmic_bytes_per_launch": alg_bytes, "ms_per_launch": ms_dec},
-        "gpu_launches": 4 * args.steps,
+        "roofline": decode_roofline(s, wl, alg_bytes, ms_dec,
+                                    measured_traffic(args.workload, args.seqs)),
+        "gpu_launches": launches * args.steps,
         "clocks": sampler.summary(),
         "e2e": e2e,
     }

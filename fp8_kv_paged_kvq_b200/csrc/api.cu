@@ -91,7 +91,7 @@ bool make_page_map(CUtensorMap* map, void* base, bool fp8, int P, int Hkv, int p
 
 constexpr int32_t kMaxBatch = kGqaMaxBatch;   // unit prefix kept in shared memory
 
-enum class Path { kNone, kGqa };
+enum class Path { kNone, kGqa, kWide };
 
 Path decode_path(const kvq_cache* c, int32_t Hq) {
   if (Hq < 1 || Hq % c->num_kv_heads) return Path::kNone;
@@ -99,12 +99,35 @@ Path decode_path(const kvq_cache* c, int32_t Hq) {
   if (c->v_pages != nullptr && c->head_dim_k == c->head_dim_v &&
       (c->head_dim_k == 64 || c->head_dim_k == 128) && c->page_size % 16 == 0 && G <= 16)
     return Path::kGqa;
+  if (c->dtype == KVQ_FP8_E4M3 && c->v_pages == nullptr && c->head_dim_k == 576 &&
+      c->head_dim_v == 512 && c->num_kv_heads == 1 && Hq == 128 &&
+      c->scale_mode == KVQ_SCALE_TOKEN && c->page_size % 64 == 0)
+    return Path::kWide;
   return Path::kNone;
 }
 
+// Persistent CTAs (8-head kernel) or CTA pairs (wide kernel).
 int32_t resolve_ctas(const kvq_cache* c, int32_t Hq, int32_t B, int32_t num_ctas) {
   if (num_ctas > 0) return num_ctas;
+  if (decode_path(c, Hq) == Path::kWide) return wide_default_pairs(B);
   return gqa_default_ctas(c->dtype == KVQ_FP8_E4M3, c->head_dim_k, Hq / c->num_kv_heads, B);
+}
+
+// 4-D map over [P][Hkv][ps][D] bytes with a (box_x bytes, box_rows, 1, 1) box.
+bool make_u8_map(CUtensorMap* map, void* base, int P, int Hkv, int ps, int D, int box_x,
+                 int box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(ps),
+                              static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(P)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(ps) * D,
+                                 static_cast<cuuint64_t>(Hkv) * ps * D};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(box_rows),
+                             1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 kvq_status decode_common(bool want_fp8, const kvq_cache* cache, const void* q, int32_t Hq,
@@ -127,7 +150,8 @@ kvq_status decode_common(bool want_fp8, const kvq_cache* cache, const void* q, i
   const int32_t ctas = resolve_ctas(cache, Hq, B, num_ctas);
   if (ctas <= 0) return KVQ_ERR_CUDA;
   const WorkspaceLayout wl =
-      workspace_layout(B, cache->num_kv_heads, Hq / cache->num_kv_heads, cache->head_dim_v, ctas);
+      workspace_layout(B, cache->num_kv_heads, Hq / cache->num_kv_heads, cache->head_dim_v, ctas,
+                       path == Path::kWide ? wide_q_image_bytes() : 0);
   if (workspace == nullptr || workspace_bytes < wl.total ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return KVQ_ERR_WORKSPACE;
@@ -146,6 +170,17 @@ kvq_status decode_common(bool want_fp8, const kvq_cache* cache, const void* q, i
   a.workspace = workspace;
   a.num_ctas = ctas;
   a.stream = static_cast<cudaStream_t>(stream);
+  if (path == Path::kWide) {
+    // key rows of one SM's 32-token half: 128-dim atoms (128-byte swizzle)
+    // and the 64-dim tail (64-byte swizzle)
+    CUtensorMap kqk, ktail;
+    if (!make_u8_map(&kqk, cache->k_pages, cache->num_pages, 1, cache->page_size, 576, 128, 32,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_u8_map(&ktail, cache->k_pages, cache->num_pages, 1, cache->page_size, 576, 64, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+      return KVQ_ERR_CUDA;
+    return from_cuda(launch_wide_decode(a, kqk, ktail));
+  }
   CUtensorMap km, vm;
   if (!make_page_map(&km, cache->k_pages, want_fp8, cache->num_pages, cache->num_kv_heads,
                      cache->page_size, cache->head_dim_k) ||
@@ -229,8 +264,9 @@ size_t kvq_decode_workspace_size(const kvq_cache* cache, int32_t B, int32_t num_
   if (B > kMaxBatch || decode_path(cache, num_q_heads) == Path::kNone) return 0;
   const int32_t ctas = resolve_ctas(cache, num_q_heads, B, num_ctas);
   if (ctas <= 0) return 0;
+  const bool wide = decode_path(cache, num_q_heads) == Path::kWide;
   return workspace_layout(B, cache->num_kv_heads, num_q_heads / cache->num_kv_heads,
-                          cache->head_dim_v, ctas)
+                          cache->head_dim_v, ctas, wide ? wide_q_image_bytes() : 0)
       .total;
 }
 

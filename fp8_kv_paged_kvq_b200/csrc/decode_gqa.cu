@@ -582,42 +582,54 @@ __global__ void __launch_bounds__(NW * 32, (NT == 1 ? 2 : 1))
 }
 
 // ---------------------------------------------------------------------------
-// Log-sum-exp combine: one block per segment (sequence, KV head).
+// Log-sum-exp combine.  Grid (segment = (sequence, KV head), head chunk): a
+// block merges the partials of up to kCombHeads query heads of one segment.
+// Warp w first turns the partial lse values of its heads into normalised
+// weights w_k = exp(lse_k - M) / sum_k exp(lse_k - M) (shared memory), then
+// the block forms out = sum_k w_k * o_k with coalesced 16-byte loads.
 // ---------------------------------------------------------------------------
 struct CombineParams {
   const int32_t* ws_pre;
   const float* ws_lse;
   const float* ws_o;
-  int32_t B, Hkv, G, Hq, Dv, num_ctas;
+  int32_t B, Hkv, G, Hq, Dv, num_ctas, heads_per_block;
   float* out;
   float* lse;
 };
 
-__global__ void __launch_bounds__(256) lse_combine_kernel(const CombineParams p) {
+constexpr int kCombThreads = 256;
+constexpr int kCombHeads = 32;        // heads per block at most
+constexpr int kMaxPieces = 64;        // partials per segment at most
+constexpr int kCombOutputs = 4096;    // outputs per block (heads_per_block * Dv) at most
+
+__global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const CombineParams p) {
   const int32_t seg = blockIdx.x;
   const int32_t b = seg / p.Hkv, h = seg - b * p.Hkv;
+  const int32_t h0 = blockIdx.y * p.heads_per_block;            // first head of this block
+  const int32_t nh = min(p.heads_per_block, p.G - h0);
   const int64_t U = p.ws_pre[p.B];
   const int32_t tiles_b = (p.ws_pre[b + 1] - p.ws_pre[b]) / p.Hkv;
-  float* out = p.out + (static_cast<int64_t>(b) * p.Hq + h * p.G) * p.Dv;
-  float* lse = p.lse ? p.lse + static_cast<int64_t>(b) * p.Hq + h * p.G : nullptr;
+  float* out = p.out + (static_cast<int64_t>(b) * p.Hq + h * p.G + h0) * p.Dv;
+  float* lse = p.lse ? p.lse + static_cast<int64_t>(b) * p.Hq + h * p.G + h0 : nullptr;
+  const int n_out = nh * p.Dv;
   if (tiles_b == 0) {
-    for (int idx = threadIdx.x; idx < p.G * p.Dv; idx += blockDim.x) out[idx] = 0.0f;
+    for (int idx = threadIdx.x; idx < n_out; idx += blockDim.x) out[idx] = 0.0f;
     if (lse)
-      for (int hh = threadIdx.x; hh < p.G; hh += blockDim.x) lse[hh] = -__int_as_float(0x7f800000);
+      for (int hh = threadIdx.x; hh < nh; hh += blockDim.x) lse[hh] = -__int_as_float(0x7f800000);
     return;
   }
   const int64_t S = p.ws_pre[b] + static_cast<int64_t>(h) * tiles_b, E = S + tiles_b;
   const int64_t N = p.num_ctas;
-  // first CTA whose range [c*U/N, (c+1)*U/N) contains unit S
-  int64_t c = S * N / U;
-  while (c + 1 < N && (c + 1) * U / N <= S) ++c;
-  while (c > 0 && c * U / N > S) --c;
-  // partial slots of the CTAs that cover part of [S, E); CTAs with an empty
-  // range (possible only when U < N) wrote nothing and are skipped
-  constexpr int kMaxPieces = 64;
   __shared__ int64_t slots[kMaxPieces];
   __shared__ int np_sh;
+  __shared__ float wts[kCombHeads][kMaxPieces];
   if (threadIdx.x == 0) {
+    // first CTA whose range [c*U/N, (c+1)*U/N) contains unit S
+    int64_t c = S * N / U;
+    while (c + 1 < N && (c + 1) * U / N <= S) ++c;
+    while (c > 0 && c * U / N > S) --c;
+    // partial slots of the CTAs that cover part of [S, E); CTAs with an empty
+    // range (possible only when U < N) wrote nothing and are skipped
     int np = 0;
     for (int64_t cc = c; cc < N && cc * U / N < E; ++cc) {
       if ((cc + 1) * U / N == cc * U / N) continue;
@@ -634,30 +646,55 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const CombineParams p)
     if (threadIdx.x == 0) atomicOr(&g_error_flags, 2u);
     return;
   }
-  for (int idx = threadIdx.x; idx < p.G * p.Dv; idx += blockDim.x) {
-    const int head = idx / p.Dv, d = idx - head * p.Dv;
-    if (np == 1) {
-      out[idx] = p.ws_o[(slots[0] * p.G + head) * p.Dv + d];
-      continue;
-    }
-    float M = -__int_as_float(0x7f800000);
-    for (int k = 0; k < np; ++k) M = fmaxf(M, p.ws_lse[slots[k] * p.G + head]);
-    float Lsum = 0.0f, O = 0.0f;
-    for (int k = 0; k < np; ++k) {
-      const float w = __expf(p.ws_lse[slots[k] * p.G + head] - M);
-      Lsum += w;
-      O += w * p.ws_o[(slots[k] * p.G + head) * p.Dv + d];
-    }
-    out[idx] = O / Lsum;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float kNegInf = -__int_as_float(0x7f800000);
+  for (int hh = warp; hh < nh; hh += kCombThreads / 32) {
+    const int head = h0 + hh;
+    const float a0 = lane < np ? p.ws_lse[slots[lane] * p.G + head] : kNegInf;
+    const float a1 = lane + 32 < np ? p.ws_lse[slots[lane + 32] * p.G + head] : kNegInf;
+    float M = fmaxf(a0, a1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float e0 = lane < np ? __expf(a0 - M) : 0.0f;
+    const float e1 = lane + 32 < np ? __expf(a1 - M) : 0.0f;
+    float L = e0 + e1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    const float inv = 1.0f / L;
+    if (lane < np) wts[hh][lane] = e0 * inv;
+    if (lane + 32 < np) wts[hh][lane + 32] = e1 * inv;
+    if (lse && lane == 0) lse[hh] = np == 1 ? a0 : M + __logf(L);
   }
-  if (lse) {
-    for (int head = threadIdx.x; head < p.G; head += blockDim.x) {
-      if (np == 1) { lse[head] = p.ws_lse[slots[0] * p.G + head]; continue; }
-      float M = -__int_as_float(0x7f800000);
-      for (int k = 0; k < np; ++k) M = fmaxf(M, p.ws_lse[slots[k] * p.G + head]);
-      float Lsum = 0.0f;
-      for (int k = 0; k < np; ++k) Lsum += __expf(p.ws_lse[slots[k] * p.G + head] - M);
-      lse[head] = M + __logf(Lsum);
+  __syncthreads();
+  // outputs in groups of four consecutive dims (Dv is a multiple of 4)
+  const int dq = p.Dv >> 2;
+  const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+  for (int i4 = threadIdx.x; i4 < nh * dq; i4 += blockDim.x) {
+    const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
+    const int head = h0 + hh;
+    float4 acc;
+    if (np == 1) {
+      acc = *reinterpret_cast<const float4*>(p.ws_o + (slots[0] * p.G + head) * p.Dv + d);
+    } else {
+      acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int k = 0; k < np; ++k) {
+        const float4 v = *reinterpret_cast<const float4*>(p.ws_o + (slots[k] * p.G + head) * p.Dv + d);
+        const float w = wts[hh][k];
+        acc.x += w * v.x;
+        acc.y += w * v.y;
+        acc.z += w * v.z;
+        acc.w += w * v.w;
+      }
+    }
+    float* dst = out + hh * p.Dv + d;
+    if (vec_out) {
+      *reinterpret_cast<float4*>(dst) = acc;
+    } else {
+      dst[0] = acc.x;
+      dst[1] = acc.y;
+      dst[2] = acc.z;
+      dst[3] = acc.w;
     }
   }
 }
@@ -665,6 +702,30 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const CombineParams p)
 // ---------------------------------------------------------------------------
 // Host side: tensor maps, occupancy, dispatch
 // ---------------------------------------------------------------------------
+cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const float* ws_o,
+                               int32_t B, int32_t Hkv, int32_t G, int32_t Hq, int32_t Dv,
+                               int32_t num_ctas, float* out, float* lse, cudaStream_t stream) {
+  CombineParams cp;
+  cp.ws_pre = ws_pre;
+  cp.ws_lse = ws_lse;
+  cp.ws_o = ws_o;
+  cp.B = B;
+  cp.Hkv = Hkv;
+  cp.G = G;
+  cp.Hq = Hq;
+  cp.Dv = Dv;
+  cp.num_ctas = num_ctas;
+  cp.out = out;
+  cp.lse = lse;
+  int hpb = kCombOutputs / (Dv > 0 ? Dv : 1);
+  hpb = hpb < 1 ? 1 : (hpb > kCombHeads ? kCombHeads : hpb);
+  cp.heads_per_block = hpb;
+  if (Dv % 4 != 0) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(B * Hkv), static_cast<unsigned>((G + hpb - 1) / hpb));
+  if (B * Hkv > 0) lse_combine_kernel<<<grid, kCombThreads, 0, stream>>>(cp);
+  return cudaGetLastError();
+}
+
 // Opt the kernel into the largest dynamic shared memory it can ask for, once
 // per device (the attribute is per function and device).
 template <bool FP8, int D, int NT, int NW, int NS>
@@ -712,20 +773,8 @@ static cudaError_t run_gqa(const DecodeArgs& a, const CUtensorMap& km, const CUt
   kern<<<a.num_ctas, K::kThreads, smem, a.stream>>>(km, vm, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CombineParams cp;
-  cp.ws_pre = p.ws_pre;
-  cp.ws_lse = p.ws_lse;
-  cp.ws_o = p.ws_o;
-  cp.B = a.B;
-  cp.Hkv = a.c.Hkv;
-  cp.G = p.G;
-  cp.Hq = a.Hq;
-  cp.Dv = a.c.Dv;
-  cp.num_ctas = a.num_ctas;
-  cp.out = a.out;
-  cp.lse = a.lse;
-  if (a.B * a.c.Hkv > 0) lse_combine_kernel<<<a.B * a.c.Hkv, 256, 0, a.stream>>>(cp);
-  return cudaGetLastError();
+  return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, a.c.Hkv, p.G, a.Hq, a.c.Dv,
+                            a.num_ctas, a.out, a.lse, a.stream);
 }
 
 // Consumer warps and pipeline depth per configuration.

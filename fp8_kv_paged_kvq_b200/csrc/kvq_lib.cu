@@ -3,5 +3,6 @@
 #include "append.cu"
 #include "validate.cu"
 #include "decode_gqa.cu"
+#include "decode_wide.cu"
 #include "api.cu"
 #include "decode_noalloc.cu"

@@ -49,7 +49,8 @@ def compare_cache(db, oc):
     assert np.array_equal(c.page_tags.cpu().numpy().view(np.uint32), oc.page_tags)
 
 
-@pytest.mark.parametrize("name,kv", [("gqa", W.FP8), ("ragged", W.FP8), ("ragged", W.BF16)])
+@pytest.mark.parametrize("name,kv", [("gqa", W.FP8), ("ragged", W.FP8), ("ragged", W.BF16),
+                                     ("wide", W.FP8)])
 def test_full_size_step(name, kv):
     spec = W.spec_by_name(name)
     spec.kv_dtype = kv
@@ -57,7 +58,8 @@ def test_full_size_step(name, kv):
     db = DecodeBatch(wl)
     if db.cache.fp8:
         db.cache.k_pages.fill_(0xCD)
-        db.cache.v_pages.fill_(0xCD)
+        if db.cache.v_pages is not None:
+            db.cache.v_pages.fill_(0xCD)
     db.prefill()
     out, lse = db.step(check_tags=True)
     torch.cuda.synchronize()

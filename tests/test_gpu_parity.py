@@ -55,6 +55,11 @@ SPECS = {
                            kv_dtype=W.BF16),
     "bf16_g12_d64": W.Spec("bf16_g12_d64", [7, 64, 333], 32, 24, 2, 64, 64, kv_dtype=W.BF16),
     "bf16_g16_d128": W.Spec("bf16_g16_d128", [100, 257], 16, 16, 1, 128, 128, kv_dtype=W.BF16),
+    # 128 query heads on one KV head, K 576 / V = first 512 dims, per-token scales
+    "wide_ps64": W.Spec("wide_ps64", [1, 63, 64, 65, 200, 700], 64, 128, 1, 576, 512,
+                        v_alias=True, scale_mode=W.SCALE_TOKEN, n_stale=1),
+    "wide_ps128": W.Spec("wide_ps128", [129, 500, 1000], 128, 128, 1, 576, 512, v_alias=True,
+                         scale_mode=W.SCALE_TOKEN),
 }
 
 
@@ -121,6 +126,60 @@ def test_split_count_sweep(num_ctas):
     torch.cuda.synchronize()
     ro, rl = OS.decode(wl, oc)
     assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), str(num_ctas))
+    assert kvq.device_error() == 0
+
+
+@pytest.mark.parametrize("num_pairs", [1, 2, 3, 7, 74, 200])
+def test_wide_split_count_sweep(num_pairs):
+    wl, db, oc = build_both(SPECS["wide_ps64"], seed=13, num_ctas=num_pairs)
+    out, lse = db.step(check_tags=False)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), str(num_pairs))
+    assert kvq.device_error() == 0
+
+
+def test_wide_outlier_query_and_peaky_scores():
+    """Queries with a wide magnitude range (the two-term E4M3 split) and a few
+    very large scores (the reference max has to move)."""
+    spec = W.Spec("wide_peaky", [300, 77], 64, 128, 1, 576, 512, v_alias=True,
+                  scale_mode=W.SCALE_TOKEN)
+    wl = W.make_workload(spec, seed=14, device="cuda")
+    q = wl.q().float()
+    q[:, :, :8] *= 40.0                       # a few large dims: peaky softmax
+    q[:, 5, :] *= 1e-3                        # a tiny-magnitude head
+    wl._q = q.to(torch.bfloat16)
+    db = DecodeBatch(wl)
+    db.prefill()
+    db.append_new()
+    oc = OS.new_cache(wl)
+    OS.fill(wl, oc)
+    out, lse = db.decode(use_abort=False)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), "peaky")
+    assert kvq.device_error() == 0
+
+
+def test_wide_out_of_range_pages_empty_and_aborted_rows():
+    """The tensor-core path: an out-of-range and a negative page inside a
+    sequence read as zero codes with zero scale, an empty sequence and an
+    aborted one give 0 / -inf, the rest match the oracle."""
+    spec = W.Spec("wide_edges", [0, 130, 64, 300, 129], 64, 128, 1, 576, 512, v_alias=True,
+                  scale_mode=W.SCALE_TOKEN)
+    wl, db, oc = build_both(spec, seed=15)
+    bt = wl.block_table.copy()
+    bt[1, 1] = wl.num_pages + 3
+    bt[3, 2] = -1
+    wl.block_table = bt
+    db.block_table = torch.from_numpy(bt).cuda()
+    abort = np.array([0, 0, 1, 0, 0], np.uint8)
+    db.abort.copy_(torch.from_numpy(abort))
+    out, lse = db.decode(use_abort=True)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc, abort=abort)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), "wide edges")
+    assert torch.all(out[[0, 2]] == 0) and torch.all(torch.isneginf(lse[[0, 2]]))
     assert kvq.device_error() == 0
 
 
