@@ -23,14 +23,19 @@
 //    E4M3 subnormal step 2^-9 (at most 2^-10 away, against a row maximum of
 //    at least 128).  A pre-pass writes both terms of every (sequence, 64-head
 //    half) as the shared-memory image the MMAs read.
-//  * One thread issues a tcgen05.mma about every 55 cycles, while an
-//    M=128, N=64, K=32 E4M3 MMA takes the tensor core about 16.  So the
-//    hi and lo chains of QK^T accumulate into two separate S buffers, each
-//    issued by its own warp, and a third warp issues PV: the three streams
-//    together keep the tensor core fed.  The softmax adds the two S terms.
+//  * One thread issues a tcgen05.mma only about every 55 cycles, and an
+//    M=128 (64 rows per SM), N=64, K=32 E4M3 MMA uses the tensor core
+//    poorly unless several are in flight.  So two warps issue: stream k
+//    takes every other 32-dim K-step of QK^T (both query terms) into its
+//    own S accumulator, then PV of the previous block for value-dim half
+//    k (N = 256).  The softmax adds the partial scores; the fixed order per
+//    stream keeps PV, which frees the P and V buffers, from queuing behind
+//    QK^T.
 //  * PV: kind::f16.  P goes to f16 with the token's scale folded in; V is
-//    converted from E4M3 to f16 (exact).  Each SM converts only the half
-//    of the 512 value dims that its half of the MMA's B operand holds.
+//    converted from E4M3 to f16 exactly, as V * 2^-8, by moving bits on the
+//    integer pipes (the conversion unit is left to exp2 and the P packing);
+//    the epilogue multiplies by 2^8.  Each SM converts only the 256 value
+//    dims that its halves of the two PV instructions' B operands hold.
 //  * The B operand of QK^T is split by tokens between the two SMs (the
 //    leader holds tokens 0-31 of the block, the other SM tokens 32-63), and
 //    both SMs' key loads complete on the leader's barrier.  The B operand of
@@ -43,10 +48,9 @@
 //    base 2 and exponentiated against a reference max that moves only when a
 //    score exceeds it by 2^8 (then O is rescaled in TMEM).
 //  * Warp roles per CTA: 0 TMA producer (three key stages, page ids read 32
-//    blocks ahead); 1 TMEM owner and QK-hi issuer; 10 QK-lo issuer; 11 PV
-//    issuer (issuers run in the leader CTA only); 2-5 softmax, P and O
-//    read-out; 6-9 V conversion.  S and converted V are double-buffered,
-//    P triple-buffered.
+//    blocks ahead); 1-2 MMA streams (leader CTA only; warp 1 also owns the
+//    tensor memory); 3-10 softmax, P and O read-out; 11-14 V conversion.
+//    S and converted V are double-buffered, P triple-buffered.
 //  * Work split as in the 8-head kernel: the pre-pass also writes the prefix
 //    of 64-token blocks over the sequences, the blocks of all sequences are
 //    split evenly over the CTA pairs (split-KV), each pair writes one
@@ -64,8 +68,15 @@ constexpr int kH = 64;     // heads per CTA
 constexpr int kDk = 576;
 constexpr int kDv = 512;
 constexpr int kBlk = 64;   // tokens per block
-constexpr int kThreads = 384;
-constexpr int kWarpQkHi = 1, kWarpQkLo = 10, kWarpPv = 11;
+#ifndef KVQ_WIDE_STREAMS
+#define KVQ_WIDE_STREAMS 2
+#endif
+constexpr int kNumMma = KVQ_WIDE_STREAMS;             // MMA streams (2 or 4)
+static_assert(kNumMma == 2 || kNumMma == 4, "MMA streams");
+constexpr int kWarpMma = 1;                           // warps 1 .. kNumMma
+constexpr int kWarpSoftmax = kWarpMma + kNumMma;      // 8 softmax warps
+constexpr int kWarpV = kWarpSoftmax + 8;              // 4 V warps
+constexpr int kThreads = 32 * (kWarpV + 4);
 
 constexpr int kNK = 3;                                // key stages
 constexpr int kQkAtom = 32 * 128;                     // 32 token rows x 128 dims
@@ -74,7 +85,7 @@ constexpr int kQAtom = 64 * 128;                      // 64 head rows x 128 dims
 constexpr int kQPart = 4 * kQAtom + 64 * 64;          // one E4M3 term: 36,864 B
 constexpr int kQImage = 2 * kQPart + kH * 4;          // hi, lo, 2^-e per head
 constexpr int kVHalf = kBlk * 128 * 2;                // 64 tokens x 128 dims f16
-constexpr int kVBuf = 2 * kVHalf;
+constexpr int kVBuf = 2 * kVHalf;                     // one CTA's 256 value dims
 constexpr int kPBuf = kH * kBlk * 2;
 constexpr int kNSc = 4;                               // scale ring entries
 constexpr int kNP = 3;                                // P buffers
@@ -86,30 +97,31 @@ constexpr int kOffP = kOffV + 2 * kVBuf;              // kNP buffers
 constexpr int kOffKSc = kOffP + kNP * kPBuf;          // token scales per key stage
 constexpr int kOffScR = kOffKSc + kNK * kBlk * 4;     // scale ring read by the softmax
 constexpr int kOffXm = kOffScR + kNSc * kBlk * 4;
-constexpr int kOffXl = kOffXm + 2 * 128 * 4;         // xm: two blocks' head maxima
-constexpr int kOffFlag = kOffXl + 128 * 4;            // per key stage: page in range
+constexpr int kOffXl = kOffXm + 2 * 256 * 4;         // xm: two blocks' partial maxima
+constexpr int kOffFlag = kOffXl + 256 * 4;            // per key stage: page in range
 constexpr int kOffBars = kOffFlag + 16;
 enum {
   // completed in the leader CTA
   kKFull = 0, kSFree = 3, kQReady = 5, kPReady = 6, kVReady = 8, kOFree = 10,
   // arrive in both CTAs (multicast commits)
-  kSHi = 11, kSLo = 13, kKFree = 15, kPvDone = 18, kPFree = 20,
+  kSFull = 11, kKFree = 13, kPvDone = 16, kPFree = 18,
   // local
-  kKPeerFull = 23, kScL = 26, kScR = 29, kQFull = 33, kDrain = 34, kNumBars = 37
+  kKPeerFull = 21, kScL = 24, kScR = 27, kQFull = 31, kDrain = 32, kNumBars = 36
 };
 constexpr int kOffTmem = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = 1024 + kOffTmem + 16;
 static_assert(kQImage <= kOffK, "query image overlaps the key stages");
 static_assert(kSmemBytes <= 232448, "shared memory");
 
-// TMEM columns: O at [0, 256) (PV instruction i at 128*i), S_hi buffers at
-// 256 + 32*s, S_lo buffers at 320 + 32*s.
+// TMEM columns: O at [0, 256) (value-dim half h of the pair at 128*h), the
+// S accumulator of MMA stream k, buffer s, at 256 + 64*k + 32*s.
+static_assert(256 + 64 * kNumMma <= 512, "tensor memory");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColSHi = 256, kColSLo = 320;
+constexpr uint32_t kColS = 256;
 
 // Instruction descriptors: FP32 accumulate (bit 4), M = 128 (m_dim = 8 at
-// bit 24), N >> 3 at bit 17; QK^T E4M3 x E4M3 both K-major; PV f16 x f16
-// with B (the values) MN-major (bit 16).
+// bit 24), N >> 3 at bit 17; QK^T E4M3 x E4M3 both K-major (N = 64 tokens);
+// PV f16 x f16 with B (the values) MN-major (bit 16), N = 256 value dims.
 constexpr uint32_t kIdescQK = (1u << 4) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
 
@@ -282,19 +294,30 @@ __device__ __forceinline__ void for_pieces(const Params& p, int32_t u0, int32_t 
   }
 }
 
-// One QK^T chain (18 MMAs of K = 32) of the query term at `sq` against key stage `sk`.
-__device__ __forceinline__ void issue_qk(uint32_t d, uint32_t sq, uint32_t sk) {
+// Stream k's share of QK^T for one block: K-steps (32 dims each) k,
+// k + kNumMma, ... of the 18, each as two MMAs (the hi and the lo query
+// term) into the stream's own S accumulator.  Each descriptor is a base plus a
+// constant in its address field (addresses stay below 256 KB, so the
+// 14-bit field cannot carry).
+__device__ __forceinline__ void issue_qk(uint32_t d, uint32_t sq, uint32_t sk, int k) {
+  const uint64_t qa = smem_desc(sq, 16, 1024, 2), ka = smem_desc(sk, 16, 1024, 2);
+  const uint64_t qt = smem_desc(sq + 4 * kQAtom, 16, 512, 4);
+  const uint64_t kt = smem_desc(sk + 4 * kQkAtom, 16, 512, 4);
+  constexpr uint64_t kLo = kQPart >> 4;                // the lo term, as a descriptor offset
 #pragma unroll
-  for (int ks = 0; ks < kDk / 32; ++ks) {
-    uint64_t ad, bd;
-    if (ks < 16) {
-      ad = smem_desc(sq + (ks >> 2) * kQAtom + (ks & 3) * 32, 16, 1024, 2);
-      bd = smem_desc(sk + (ks >> 2) * kQkAtom + (ks & 3) * 32, 16, 1024, 2);
-    } else {
-      ad = smem_desc(sq + 4 * kQAtom + (ks - 16) * 32, 16, 512, 4);
-      bd = smem_desc(sk + 4 * kQkAtom + (ks - 16) * 32, 16, 512, 4);
+  for (int t = 0; t < (18 + kNumMma - 1) / kNumMma; ++t) {
+    const int ks = k + kNumMma * t;
+    if (ks < 16) {                           // dims 0..511: 128-byte-swizzled atoms
+      const uint64_t qo = qa + (((ks >> 2) * kQAtom + (ks & 3) * 32) >> 4);
+      const uint64_t ko = ka + (((ks >> 2) * kQkAtom + (ks & 3) * 32) >> 4);
+      umma_pair_f8(d, qo, ko, kIdescQK, t > 0 ? 1u : 0u);
+      umma_pair_f8(d, qo + kLo, ko, kIdescQK, 1u);
+    } else if (ks < 18) {                    // dims 512..575: the 64-byte-swizzled tail
+      const uint64_t qo = qt + (((ks - 16) * 32) >> 4);
+      const uint64_t ko = kt + (((ks - 16) * 32) >> 4);
+      umma_pair_f8(d, qo, ko, kIdescQK, 1u);
+      umma_pair_f8(d, qo + kLo, ko, kIdescQK, 1u);
     }
-    umma_pair_f8(d, ad, bd, kIdescQK, ks > 0 ? 1u : 0u);
   }
 }
 
@@ -313,27 +336,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNK; ++s) {
       mbar_init(&bars[kKFull + s], 1);
-      mbar_init(&bars[kKFree + s], 4);        // two QK chains + both CTAs' V conversion
+      mbar_init(&bars[kKFree + s], kNumMma + 8);   // the MMA streams + both CTAs' four V warps
       mbar_init(&bars[kKPeerFull + s], 1);
       mbar_init(&bars[kScL + s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars[kSFree + s], 2);
-      mbar_init(&bars[kPReady + s], 2);
-      mbar_init(&bars[kVReady + s], 2);
-      mbar_init(&bars[kSHi + s], 1);
-      mbar_init(&bars[kSLo + s], 1);
-      mbar_init(&bars[kPvDone + s], 1);
+      mbar_init(&bars[kSFree + s], 16);       // per softmax warp, both CTAs
+      mbar_init(&bars[kPReady + s], 16);
+      mbar_init(&bars[kVReady + s], 8);
+      mbar_init(&bars[kSFull + s], kNumMma);  // one commit per MMA stream
+      mbar_init(&bars[kPvDone + s], kNumMma);
     }
-    for (int s = 0; s < kNP; ++s) mbar_init(&bars[kPFree + s], 1);
+    for (int s = 0; s < kNP; ++s) mbar_init(&bars[kPFree + s], kNumMma);
     for (int s = 0; s < kNSc; ++s) mbar_init(&bars[kScR + s], 1);
     mbar_init(&bars[kQReady], 2);
-    mbar_init(&bars[kOFree], 2);
+    mbar_init(&bars[kOFree], 16);
     mbar_init(&bars[kQFull], 1);
-    for (int s = 0; s < 3; ++s) mbar_init(&bars[kDrain + s], 1);
+    for (int s = 0; s < kNumMma; ++s) mbar_init(&bars[kDrain + s], 1);
     fence_barrier_init();
   }
-  if (warp == kWarpQkHi) {
+  if (warp == kWarpMma) {
     tmem_alloc_pair(tmem_slot, kTmemCols);
     tmem_relinquish_pair();
     tc_fence_before();
@@ -413,75 +435,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_cluster(&bars[kScL + j % kNK], ph);
       }
     }
-  } else if (warp == kWarpQkHi || warp == kWarpQkLo) {
-    // ---------------- QK^T issue, one E4M3 term per warp (leader CTA) ----------------
+  } else if (warp < kWarpMma + kNumMma) {
+    // ---------------- MMA issue, kNumMma streams (leader CTA) ----------------
+    // Stream k issues its share of QK^T for block j, then (streams 0 and 1)
+    // PV of block j-1 for value-dim half k.  A thread issues a
+    // tcgen05.mma only about every 55 cycles, so several streams keep the
+    // tensor core fed; the fixed order per stream keeps PV (which frees the
+    // P and V buffers) from queuing behind QK^T.
     if (rank == 0 && lane == 0) {
-      const int part = warp == kWarpQkLo ? 1 : 0;
-      const uint32_t sq = smem_u32(smem + kOffQ) + part * kQPart;
-      const uint32_t sk = smem_u32(smem + kOffK);
-      const uint32_t dcol = tbase + (part ? kColSLo : kColSHi);
-      uint64_t* s_full = &bars[part ? kSLo : kSHi];
+      const int k = warp - kWarpMma;
+      const uint32_t sq = smem_u32(smem + kOffQ), sk = smem_u32(smem + kOffK);
+      const uint32_t sv = smem_u32(smem + kOffV), sp = smem_u32(smem + kOffP);
+      const uint32_t dcol = tbase + kColS + 64 * k;
       int32_t j = 0, item = 0;
       bool ok = true;
+      // PV of block jj, value-dim half h = k (dims 256h + [0, 256) across
+      // the pair) into O columns [128h, 128h + 128); streams 2, 3 have none
+      auto pv = [&](int32_t jj, bool first) {
+        const int x = jj & 1;
+        const uint32_t ph = (jj >> 1) & 1;
+        ok = ok && wait_bar(&bars[kPReady + x], ph) && wait_bar(&bars[kVReady + x], ph);
+        if (ok && first && item > 0) ok = wait_bar(&bars[kOFree], (item - 1) & 1);
+        if (!ok) return;
+        tc_fence_after();
+        const uint64_t pa = smem_desc(sp + (jj % kNP) * kPBuf, 16, 1024, 2);
+        if (k < 2) {
+          const uint64_t va = smem_desc(sv + x * kVBuf + k * kVHalf, 1024, 2048, 2);
+#pragma unroll
+          for (int ks = 0; ks < kBlk / 16; ++ks)
+            umma_pair_f16(tbase + 128 * k, pa + ((ks * 32) >> 4), va + ((ks * 4096) >> 4),
+                          kIdescPV, (first && ks == 0) ? 0u : 1u);
+        }
+        umma_commit_pair(&bars[kPvDone + x]);
+        umma_commit_pair(&bars[kPFree + jj % kNP]);
+      };
       for_pieces(p, u0, u1, [&](int, int32_t, int32_t nt) {
         ok = ok && wait_bar(&bars[kQReady], item & 1);
         for (int32_t i = 0; i < nt && ok; ++i, ++j) {
           const int s = j % kNK, s2 = j & 1;
           ok = wait_bar(&bars[kKFull + s], static_cast<uint32_t>(j / kNK) & 1u);
-          if (ok && part == 0)     // the other CTA's V conversion learns that both stages landed
+          if (ok && k == 0)        // the other CTA's V conversion learns that both stages landed
             mbar_arrive_remote(mapa_shared(smem_u32(&bars[kKPeerFull + s]), 1));
           if (ok && j >= 2) ok = wait_bar(&bars[kSFree + s2], ((j >> 1) & 1) ^ 1);
           if (!ok) break;
           tc_fence_after();
-          issue_qk(dcol + 32 * s2, sq, sk + s * kStage);
-          umma_commit_pair(&s_full[s2]);
+          issue_qk(dcol + 32 * s2, sq, sk + s * kStage, k);
+          umma_commit_pair(&bars[kSFull + s2]);
           umma_commit_pair(&bars[kKFree + s]);
+          if (i > 0) pv(j - 1, i == 1);
         }
+        if (ok && nt > 0) pv(j - 1, nt == 1);
         ++item;
       });
       // every MMA issued has finished before either CTA leaves
-      umma_commit_pair_local(&bars[kDrain + part]);
-      mbar_wait_cluster(&bars[kDrain + part], 0);
+      umma_commit_pair_local(&bars[kDrain + k]);
+      mbar_wait_cluster(&bars[kDrain + k], 0);
     }
-  } else if (warp == kWarpPv) {
-    // ---------------- PV issue (leader CTA) ----------------
-    if (rank == 0 && lane == 0) {
-      const uint32_t sv = smem_u32(smem + kOffV), sp = smem_u32(smem + kOffP);
-      int32_t j = 0, item = 0;
-      bool ok = true;
-      for_pieces(p, u0, u1, [&](int, int32_t, int32_t nt) {
-        for (int32_t i = 0; i < nt && ok; ++i, ++j) {
-          const int x = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          ok = wait_bar(&bars[kPReady + x], ph) && wait_bar(&bars[kVReady + x], ph);
-          if (ok && i == 0 && item > 0) ok = wait_bar(&bars[kOFree], (item - 1) & 1);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t spj = sp + (j % kNP) * kPBuf;
-#pragma unroll
-          for (int ks = 0; ks < kBlk / 16; ++ks)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-              const uint64_t a = smem_desc(spj + ks * 32, 16, 1024, 2);
-              const uint64_t bd =
-                  smem_desc(sv + x * kVBuf + hf * kVHalf + ks * 4096, 1024, 2048, 2);
-              umma_pair_f16(tbase + 128 * hf, a, bd, kIdescPV, (i == 0 && ks == 0) ? 0u : 1u);
-            }
-          umma_commit_pair(&bars[kPvDone + x]);
-          umma_commit_pair(&bars[kPFree + j % kNP]);
-        }
-        ++item;
-      });
-      umma_commit_pair_local(&bars[kDrain + 2]);
-      mbar_wait_cluster(&bars[kDrain + 2], 0);
-    }
-  } else if (warp >= 6) {
+  } else if (warp >= kWarpV) {
     // ---------------- V conversion: E4M3 codes -> f16 B operand of PV ----------------
-    const int vt = threadIdx.x - 192;                     // 0..127
-    const int tt = vt & 63, vh = vt >> 6;                 // token, PV instruction half
+    const int vt = threadIdx.x - 32 * kWarpV;             // 0..127
+    const int tt = vt & 63, vh = vt >> 6;                 // token, PV half
     const int row = tt & 31;
-    // token tt sits in the key stage of CTA tt / 32; this CTA's value dims
-    // 256*vh + 128*rank + [0, 128) are atom 2*vh + rank of that stage
+    // Token tt sits in the key stage of CTA tt / 32.  PV half h covers value
+    // dims 256h + [0, 256); this CTA holds dims 256h + 128*rank + [0, 128),
+    // the stage's 128-dim atom 2h + rank.  This thread converts half vh.
     const uint32_t src = mapa_shared(smem_u32(smem + kOffK), static_cast<uint32_t>(tt >> 5)) +
                          (2 * vh + rank) * kQkAtom;
     const float* kscl = reinterpret_cast<const float*>(smem + kOffKSc);
@@ -497,61 +514,93 @@ __global__ void __launch_bounds__(kThreads, 1)
         // loads, and the leader's QK-hi issuer forwards its completion
         ok = ok && wait_bar(&bars[rank == 0 ? kKFull + s : kKPeerFull + s], n & 1u);
         ok = ok && wait_bar(&bars[kScL + s], n & 1u);
+        const int32_t nvalid = min(kBlk, ntok - (t0 + i) * kBlk);
+        if (vt < 32) {
+          // token scales for the softmax first (0 past the end or off the
+          // cache), so the softmax never waits for the conversion below
+          if (ok) {
+            const bool in = flag[s] != 0;
+            const float2 sv = reinterpret_cast<const float2*>(kscl + s * kBlk)[vt];
+            reinterpret_cast<float2*>(ring + (j & (kNSc - 1)) * kBlk)[vt] =
+                make_float2(in && 2 * vt < nvalid ? sv.x : 0.0f, in && 2 * vt + 1 < nvalid ? sv.y : 0.0f);
+          }
+          __syncwarp();
+          if (vt == 0 && ok) mbar_arrive(&bars[kScR + (j & (kNSc - 1))]);
+        }
+        // Load and convert the codes into registers, then hand the key stage
+        // back at once; only the stores wait for the converted-V buffer.
+        const bool valid = ok && tt < nvalid;
+        const uint32_t sa = src + s * kStage;
+        uint4 wv[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          wv[c] = valid ? ld_cluster128(sa + sw128(row, c)) : make_uint4(0, 0, 0, 0);
+        uint32_t f[8][8];                                 // values * 2^-8 (undone in the epilogue)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {                     // 16 codes = dims 16c..16c+15
+          e4m3x4_to_f16x2x2_shr8(wv[c].x, f[c][0], f[c][1]);
+          e4m3x4_to_f16x2x2_shr8(wv[c].y, f[c][2], f[c][3]);
+          e4m3x4_to_f16x2x2_shr8(wv[c].z, f[c][4], f[c][5]);
+          e4m3x4_to_f16x2x2_shr8(wv[c].w, f[c][6], f[c][7]);
+        }
+        // The conversions above read every loaded register, so once they have
+        // run (the empty asm pins them before the arrivals) this thread's
+        // loads from both stages have returned; the warp sync covers all lanes.
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          asm volatile("" ::"r"(f[c][0]), "r"(f[c][1]), "r"(f[c][2]), "r"(f[c][3]), "r"(f[c][4]),
+                       "r"(f[c][5]), "r"(f[c][6]), "r"(f[c][7]));
+        __syncwarp();
+        if (lane == 0 && ok) {
+          mbar_arrive(&bars[kKFree + s]);
+          mbar_arrive_remote(mapa_shared(smem_u32(&bars[kKFree + s]), rank ^ 1u));
+        }
         if (j >= 2) ok = ok && wait_bar(&bars[kPvDone + x], ((j >> 1) & 1) ^ 1);
         if (ok) {
-          const int32_t nvalid = min(kBlk, ntok - (t0 + i) * kBlk);
-          const bool valid = tt < nvalid;
-          const uint32_t sa = src + s * kStage;
+          // MN-major, 128-byte swizzle: atoms of 64 dims x 8 tokens (1 KB),
+          // two atoms per 8 tokens
           uint8_t* dst = smem + kOffV + x * kVBuf + vh * kVHalf;
-          uint4 wv[8];                                    // all eight loads in flight at once
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            wv[c] = valid ? ld_cluster128(sa + sw128(row, c)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {                   // 16 codes = dims 16c..16c+15
-            const uint4 w = wv[c];
-            uint32_t f[8];
-            e4m3x4_to_f16x2x2(w.x, f[0], f[1]);
-            e4m3x4_to_f16x2x2(w.y, f[2], f[3]);
-            e4m3x4_to_f16x2x2(w.z, f[4], f[5]);
-            e4m3x4_to_f16x2x2(w.w, f[6], f[7]);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {              // 8 dims per 16-byte V chunk
               const int cc = 2 * c + hh;
               const uint32_t off = (cc >> 3) * 1024 + (tt >> 3) * 2048 + (tt & 7) * 128 +
                                    (((cc & 7) ^ (tt & 7)) << 4);
-              *reinterpret_cast<uint4*>(dst + off) =
-                  make_uint4(f[4 * hh], f[4 * hh + 1], f[4 * hh + 2], f[4 * hh + 3]);
+              *reinterpret_cast<uint4*>(dst + off) = make_uint4(
+                  f[c][4 * hh], f[c][4 * hh + 1], f[c][4 * hh + 2], f[c][4 * hh + 3]);
             }
-          }
-          if (vt < kBlk)      // token scales for the softmax (0 past the end or off the cache)
-            ring[(j & (kNSc - 1)) * kBlk + vt] = (flag[s] != 0 && vt < nvalid) ? kscl[s * kBlk + vt] : 0.0f;
         }
         fence_proxy_async_smem();
-        named_bar(2, 128);
-        if (vt == 0 && ok) {      // the softmax and the PV issuer first, then the stage
-          mbar_arrive(&bars[kScR + (j & (kNSc - 1))]);
-          arrive_leader(&bars[kVReady + x], rank);
-          mbar_arrive(&bars[kKFree + s]);
-          mbar_arrive_remote(mapa_shared(smem_u32(&bars[kKFree + s]), rank ^ 1u));
-        }
+        __syncwarp();
+        if (lane == 0 && ok) arrive_leader(&bars[kVReady + x], rank);   // per warp
       }
     });
   } else {
     // ---------------- softmax warps: scores, P, epilogue ----------------
-    const int mt = threadIdx.x - 64;                      // 0..127
-    const int L = 32 * (warp & 3) + lane;                 // this thread's TMEM lane
+    // Eight warps.  Warp w reads TMEM lane quarter q = w % 4 (lane L = 32q +
+    // lane: head L % 64, token half L / 64) and column half ch of the block's
+    // 32 columns per lane, i.e. tokens 32*(L/64) + 16*ch + [0, 16).  The four
+    // warps holding the same 32 heads (quarters q and q^2, both column
+    // halves) exchange partial maxima and sums through shared memory.
+    const int mt = threadIdx.x - 32 * kWarpSoftmax;       // 0..255
+    const int q4 = warp & 3, ch = (warp - kWarpSoftmax) >> 2;
+    const int L = 32 * q4 + lane;                         // this thread's TMEM lane
     const int hl = L & 63, half = L >> 6;                 // head (in this CTA), token half
-    const uint32_t tl = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    const int part = 2 * half + ch;                       // which 16 of the head's 64 tokens
+    const uint32_t tl = tbase + (static_cast<uint32_t>(32 * q4) << 16);
     const float* qexp = reinterpret_cast<const float*>(smem + kOffQ + 2 * kQPart);
     const float* ring = reinterpret_cast<const float*>(smem + kOffScR);
     float* xm = reinterpret_cast<float*>(smem + kOffXm);
     float* xl = reinterpret_cast<float*>(smem + kOffXl);
     const float kNegInf = -__int_as_float(0x7f800000);
+    const uint32_t group_bar = 3 + (warp & 1);            // the four warps of these heads
     int32_t j = 0, item = 0, q_loads = 0;
     bool ok = true;
-    // Every softmax thread runs the same loop trips and named barriers; after
-    // a failed wait (ok == false) the work is skipped but the barriers kept.
+    // Every softmax thread runs the same loop trips and barriers; after a
+    // failed wait (ok == false) the work is skipped but the barriers kept.
+    // Each warp reports to the MMA issuers on its own (counts of 16: eight
+    // warps in each CTA).
     for_pieces(p, u0, u1, [&](int b, int32_t t0, int32_t nt) {
       const int32_t ntok = seq_tokens(p, b);
       // ---- this CTA's half of the query image (the previous piece's QK^T
@@ -566,33 +615,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ok = ok && wait_bar(&bars[kQFull], item & 1);
       if (mt == 0 && ok) arrive_leader(&bars[kQReady], rank);
+      // read once: the next piece's image load (by thread 0 after its last
+      // PV, which needs every warp's last P) may overwrite it
+      const float alpha = p.sm_scale * kLog2e * qexp[hl];
 
       float m_ref = kNegInf, l_part = 0.0f;
       for (int32_t i = 0; i < nt; ++i, ++j) {
         const int s2 = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         const int32_t nvalid = min(kBlk, ntok - (t0 + i) * kBlk);
-        ok = ok && wait_bar(&bars[kSHi + s2], ph) && wait_bar(&bars[kSLo + s2], ph);
+        ok = ok && wait_bar(&bars[kSFull + s2], ph);
         ok = ok && wait_bar(&bars[kScR + (j & (kNSc - 1))], (j >> 2) & 1);
         ok = __all_sync(0xffffffffu, ok);                   // tcgen05.ld is warp-collective
         tc_fence_after();
-        uint32_t rh[32], rl[32];
+        // the streams' partial scores (each covers its share of the dims)
+        float sacc[16];
         if (ok) {
-          tmem_ld32(tl + kColSHi + 32 * s2, rh);
-          tmem_ld32(tl + kColSLo + 32 * s2, rl);
-          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) sacc[c] = 0.0f;
+#pragma unroll
+          for (int k2 = 0; k2 < kNumMma; k2 += 2) {
+            uint32_t r0[16], r1[16];
+            tmem_ld16(tl + kColS + 64 * k2 + 32 * s2 + 16 * ch, r0);
+            tmem_ld16(tl + kColS + 64 * (k2 + 1) + 32 * s2 + 16 * ch, r1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) sacc[c] += __uint_as_float(r0[c]) + __uint_as_float(r1[c]);
+          }
         } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) rh[c] = rl[c] = 0u;
+          for (int c = 0; c < 16; ++c) sacc[c] = 0.0f;
         }
         tc_fence_before();
-        // this thread's 32 token scales (0 past the end of the sequence or off the cache)
-        float sc[32];
+        // this thread's 16 token scales (0 past the end of the sequence or off the cache)
+        float sc[16];
         {
-          const float4* s4 =
-              reinterpret_cast<const float4*>(ring + (j & (kNSc - 1)) * kBlk + 32 * half);
+          const float4* s4 = reinterpret_cast<const float4*>(ring + (j & (kNSc - 1)) * kBlk + 16 * part);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
+          for (int k = 0; k < 4; ++k) {
             const float4 v = s4[k];
             sc[4 * k] = v.x;
             sc[4 * k + 1] = v.y;
@@ -600,29 +660,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             sc[4 * k + 3] = v.w;
           }
         }
-        const float alpha = p.sm_scale * kLog2e * qexp[hl];
-        float x[32];
+        float x[16];
         float bm = kNegInf;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] = (__uint_as_float(rh[c]) + __uint_as_float(rl[c])) * (alpha * sc[c]);
+        for (int c = 0; c < 16; ++c)
+          x[c] = sacc[c] * (alpha * sc[c]);
         if (nvalid < kBlk) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (32 * half + c >= nvalid) x[c] = kNegInf;
+          for (int c = 0; c < 16; ++c)
+            if (16 * part + c >= nvalid) x[c] = kNegInf;
         }
 #pragma unroll
-        for (int c = 0; c < 32; ++c) bm = fmaxf(bm, x[c]);
-        // head maxima, double-buffered by block parity: the next write to this
-        // half comes after the next block's barrier, which the partner passes
-        // only after this read
-        float* xmj = xm + s2 * 128;
-        xmj[L] = bm;
-        named_bar(1, 128);                                // every S load of this block done
-        if (mt == 0 && ok) arrive_leader(&bars[kSFree + s2], rank);
-        bm = fmaxf(bm, xmj[L ^ 64]);
+        for (int c = 0; c < 16; ++c) bm = fmaxf(bm, x[c]);
+        // partial maxima, double-buffered by block parity: the next write to
+        // this buffer comes after the next block's barrier, which the other
+        // three warps pass only after this block's reads
+        float* xmj = xm + s2 * 256;
+        xmj[part * 64 + hl] = bm;
+        named_bar(group_bar, 128);                        // this warp's S loads are done too
+        if (lane == 0 && ok) arrive_leader(&bars[kSFree + s2], rank);
+#pragma unroll
+        for (int o = 1; o < 4; ++o) bm = fmaxf(bm, xmj[((part + o) & 3) * 64 + hl]);
         // Move the reference max when a score exceeds it by 2^8.  The vote keeps
-        // the TMEM accesses warp-uniform; the warp holding the other token half
-        // of the same 32 heads sees the same head maxima and votes alike.
+        // the TMEM accesses warp-uniform; the other three warps of these 32
+        // heads see the same head maxima and vote alike.
         if (__any_sync(0xffffffffu, bm > m_ref + 8.0f)) {
           const float m_new = fmaxf(m_ref, bm);
           const float r = ex2(m_ref - m_new);             // 0 on the first block, 1 if unmoved
@@ -632,9 +693,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = ok && wait_bar(&bars[kPvDone + ((j - 1) & 1)], ((j - 1) >> 1) & 1);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            if (ok) {
+            if (ok) {                                     // this warp's half of O's columns
 #pragma unroll 1
-              for (int cc = 0; cc < 8; ++cc) {
+              for (int cc = 4 * ch; cc < 4 * ch + 4; ++cc) {
                 uint32_t o[32];
                 tmem_ld32(tl + 32 * cc, o);
                 tmem_wait_ld();
@@ -648,9 +709,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_ref = m_new;
         }
         // ---- P (f16, token scale folded in) into the A operand of PV ----
-        uint32_t pk[16];
+        uint32_t pk[8];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < 16; c += 2) {
           const float p0 = ex2(x[c] - m_ref), p1 = ex2(x[c + 1] - m_ref);
           l_part += p0 + p1;
           pk[c >> 1] = pack_f16x2(p0 * sc[c], p1 * sc[c + 1]);
@@ -660,14 +721,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = ok && wait_bar(&bars[kPFree + pb], static_cast<uint32_t>((j / kNP) & 1) ^ 1u);
         if (ok) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(smem + kOffP + pb * kPBuf + sw128(hl, 4 * half + k)) =
+          for (int k = 0; k < 2; ++k)
+            *reinterpret_cast<uint4*>(smem + kOffP + pb * kPBuf + sw128(hl, 2 * part + k)) =
                 make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
         tc_fence_before();
         fence_proxy_async_smem();
-        named_bar(1, 128);
-        if (mt == 0 && ok) arrive_leader(&bars[kPReady + s2], rank);
+        __syncwarp();
+        if (lane == 0 && ok) arrive_leader(&bars[kPReady + s2], rank);
       }
 
       // ---- epilogue: O / l and lse for this piece ----
@@ -676,18 +737,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = ok && wait_bar(&bars[kPvDone + (jl & 1)], (jl >> 1) & 1);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
-        xl[L] = l_part;
-        named_bar(1, 128);
-        const float l_tot = l_part + xl[L ^ 64];
-        const float inv = 1.0f / l_tot;
+        xl[part * 64 + hl] = l_part;
+        named_bar(group_bar, 128);
+        float l_tot = l_part;
+#pragma unroll
+        for (int o = 1; o < 4; ++o) l_tot += xl[((part + o) & 3) * 64 + hl];
+        const float inv = 256.0f / l_tot;                 // V was converted as V * 2^-8
         const int hg = 64 * static_cast<int>(rank) + hl;
         const int64_t slot = pair + b;
         float* orow = p.ws_o + (slot * kHq + hg) * kDv;
 #pragma unroll 1
-        for (int cc = 0; cc < 8 && ok; ++cc) {
+        for (int cc = 4 * ch; cc < 4 * ch + 4 && ok; ++cc) {
           uint32_t o[32];
           tmem_ld32(tl + 32 * cc, o);
           tmem_wait_ld();
+          // column 32*cc: value-dim half cc/4, this lane half's 128 dims
           const int dv0 = 256 * (cc >> 2) + 128 * half + 32 * (cc & 3);
 #pragma unroll
           for (int k = 0; k < 32; k += 4)
@@ -695,10 +759,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_float4(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv,
                             __uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
         }
-        if (half == 0 && ok) p.ws_lse[slot * kHq + hg] = (m_ref + __log2f(l_tot)) * kLn2;
+        if (part == 0 && ok) p.ws_lse[slot * kHq + hg] = (m_ref + __log2f(l_tot)) * kLn2;
         tc_fence_before();
-        named_bar(1, 128);
-        if (mt == 0 && ok) arrive_leader(&bars[kOFree], rank);
+        // xl is rewritten at the next piece's epilogue, after many group barriers
+        __syncwarp();
+        if (lane == 0 && ok) arrive_leader(&bars[kOFree], rank);
       }
       ++item;
     });
@@ -708,7 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   __syncthreads();
   cluster_sync_all();            // the leader's MMAs no longer read this CTA's memory
-  if (warp == kWarpQkHi) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc_pair(tbase, kTmemCols);
   }

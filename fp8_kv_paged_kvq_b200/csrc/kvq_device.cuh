@@ -188,6 +188,19 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint
       : "r"(w));
 }
 
+// Four E4M3 codes to two f16x2 holding each value times 2^-8, with bit moves
+// only (no conversion unit).  An E4M3 code s.eeee.mmm placed at f16 bits
+// s -> 15, eeee.mmm -> 13..7 is the same number scaled by 2^(7-15) = 2^-8:
+// the f16 format has one more exponent bit and seven more mantissa bits, so
+// this holds for subnormal codes as well.  The NaN codes 0x7F / 0xFF come
+// out as +-480 * 2^-8.  Bytes 0,1 -> lo, bytes 2,3 -> hi.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2_shr8(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t a = prmt(w, 0u, 0x4140u) << 7;   // codes 0, 1 in the 16-bit lanes, shifted
+  const uint32_t b = prmt(w, 0u, 0x4342u) << 7;   // codes 2, 3
+  lo = a + (a & 0x40004000u);                      // carry each sign bit from 14 up to 15
+  hi = b + (b & 0x40004000u);
+}
+
 // Two floats to one packed pair of E4M3 codes (a -> low byte), rounding to
 // nearest even with saturation to +-448 (NaN -> NaN code).
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
@@ -325,9 +338,9 @@ __device__ __forceinline__ void umma_pair_f8(uint32_t d_tmem, uint64_t a_desc, u
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;"
       "\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u)
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void umma_pair_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -335,9 +348,9 @@ __device__ __forceinline__ void umma_pair_f16(uint32_t d_tmem, uint64_t a_desc, 
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;"
       "\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u)
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -397,6 +410,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[31])
       : "r"(taddr));
 }
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
