@@ -502,61 +502,70 @@ def run_long(args):
         sampler = ClockSampler(local)
         with sampler:
             for ls in W.loop_steps(wl, steps):
-                kind = ls.step % 3          # 0: check + stale tags, 1: clean check, 2: no check
+                # kind 0: check + stale tags, 1: clean check, 2: no check; the
+                # second half of each six-step cycle replays the graphs with
+                # events between the kernels, for the per-kernel breakdown
+                kind = ls.step % 3
+                detailed = (ls.step // 3) % 2 == 1
                 chk = kind != 2
                 idx = loop.prepare(ls, chk, inject_stale=(kind == 0))
-                ev = loop.run(chk, stream)
+                ev = loop.run(chk, stream, detailed)
                 loop.restore(idx)
                 torch.cuda.synchronize()
-                t_app, t_val, t_dec = (ev[i].elapsed_time(ev[i + 1]) for i in range(3))
+                ms_step = ev[0].elapsed_time(ev[-1])
+                parts = tuple(ev[i].elapsed_time(ev[i + 1]) for i in range(3)) if detailed else (0, 0, 0)
                 aborted = {b for b, _ in ls.stale} if kind == 0 else set()
                 kv = sum(int(ls.seq_lens[b]) for b in range(spec.B) if b not in aborted) * row
-                recs.append((kind, t_app, t_val, t_dec, kv, len(aborted)))
+                recs.append((kind, detailed, ms_step) + parts + (kv, len(aborted)))
     assert kvq.device_error() == 0, "device-side wait timed out"
     kind = np.array([r[0] for r in recs])
-    t_app = np.array([r[1] for r in recs])
-    t_val = np.array([r[2] for r in recs])
-    t_dec = np.array([r[3] for r in recs])
-    kv = np.array([r[4] for r in recs], dtype=np.float64)
-    ms = t_app + t_val + t_dec
+    det = np.array([r[1] for r in recs])
+    ms = np.array([r[2] for r in recs])
+    t_app = np.array([r[3] for r in recs])
+    t_val = np.array([r[4] for r in recs])
+    t_dec = np.array([r[5] for r in recs])
+    kv = np.array([r[6] for r in recs], dtype=np.float64)
     # the tracker's view must match what the device did
     host_tags = loop.tracker.tags
     dev_tags = loop.batch.cache.page_tags.cpu().numpy().view(np.uint32)
     tags_ok = bool(np.array_equal(host_tags, dev_tags))
     def mean(x):
         return float(max_over_ranks(float(np.mean(x)), world))
-    step_clean, step_nochk = mean(ms[kind == 1]), mean(ms[kind == 2])
-    # the no-check graph records the same events around an empty slot: its gap is
-    # the event overhead, subtracted from the validate slot
-    val = mean(t_val[kind == 1]) - mean(t_val[kind == 2])
-    gbs = world * kv.sum() / (max_over_ranks(float(ms.sum()), world) * 1e-3) / 1e9
+    plain = ~det                                  # steps timed only at their boundaries
+    step_clean, step_nochk = mean(ms[plain & (kind == 1)]), mean(ms[plain & (kind == 2)])
+    # in the detailed graphs the no-check step records the same events around an
+    # empty slot: its gap is the event overhead, subtracted from the validate slot
+    val = mean(t_val[det & (kind == 1)]) - mean(t_val[det & (kind == 2)])
+    gbs = world * kv[plain].sum() / (max_over_ranks(float(ms[plain].sum()), world) * 1e-3) / 1e9
     hbm, hbm_kind = peaks()
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
-        "warmup": 1, "ms_per_step": float(ms.mean()), "higher_is_better": True,
+        "warmup": 1, "ms_per_step": float(ms[plain].mean()), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "f16 mma / f32 accumulate (e4m3 cache)", "data": "synthetic",
         "config": {"workload": workload_desc("long"),
                    "loop": f"{steps} steps: append 1 token/seq with page reallocation + tag "
                            "bump; steps cycle validate+stale tags / validate / no validation",
                    "l2": "inputs exceed L2: >3 GB of cache read per step",
-                   "timing": "CUDA graph per step between CUDA events"},
-        "decode_tokens_per_s": world * spec.B / (ms.mean() * 1e-3),
+                   "timing": "CUDA graph per step between CUDA events; step time and value "
+                             "from the half of the steps with events only around the step"},
+        "decode_tokens_per_s": world * spec.B / (ms[plain].mean() * 1e-3),
         "hbm_frac_of_step": gbs / world / hbm,
         "ms_per_step_with_validation": step_clean,
         "ms_per_step_without_validation": step_nochk,
-        "ms_per_step_with_validation_and_stale_tags": mean(ms[kind == 0]),
-        "p95_ms_with_validation": float(np.percentile(ms[kind == 1], 95)),
-        "p95_ms_without_validation": float(np.percentile(ms[kind == 2], 95)),
+        "ms_per_step_with_validation_and_stale_tags": mean(ms[plain & (kind == 0)]),
+        "p95_ms_with_validation": float(np.percentile(ms[plain & (kind == 1)], 95)),
+        "p95_ms_without_validation": float(np.percentile(ms[plain & (kind == 2)], 95)),
         "ms_validate_kernel": val,
-        "ms_decode_with_validation": mean(t_dec[kind == 1]),
-        "ms_decode_without_validation": mean(t_dec[kind == 2]),
-        "ms_decode_with_stale_aborts": mean(t_dec[kind == 0]),
-        "ms_append": mean(t_app),
+        "ms_decode_with_validation": mean(t_dec[det & (kind == 1)]),
+        "ms_decode_without_validation": mean(t_dec[det & (kind == 2)]),
+        "ms_decode_with_stale_aborts": mean(t_dec[det & (kind == 0)]),
+        "ms_append": mean(t_app[det]),
         "validate_overhead_pct": 100.0 * (step_clean - step_nochk) / step_nochk,
         "validate_overhead_note": "steps cycle: validate with 0.01% stale tags / validate with "
-                                  "clean tags / no validation; overhead compares the last two",
-        "aborted_requests_per_stale_step": float(np.mean([r[5] for r in recs if r[0] == 0])),
+                                  "clean tags / no validation; overhead compares the last two, "
+                                  "each timed only at the step's boundaries",
+        "aborted_requests_per_stale_step": float(np.mean([r[7] for r in recs if r[0] == 0])),
         "pages_reallocated": int(sum(len(l.new_pages) for l in W.loop_steps(wl, steps))),
         "host_tracker_matches_device_tags": tags_ok,
         "clocks": sampler.summary(), "gpu_launches": int(4 * np.sum(kind != 2) + 3 * np.sum(kind == 2)),

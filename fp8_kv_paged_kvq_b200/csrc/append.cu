@@ -123,6 +123,7 @@ struct AppendArgs {
 constexpr int kAppendWarps = 8;
 
 __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a) {
+  pdl_trigger();            // the tag check may start loading its block-table entries
   const CacheView& c = a.c;
   if (static_cast<int32_t>(blockIdx.x) >= a.token_blocks) {
     for (int32_t i = threadIdx.x; i < a.n_realloc; i += blockDim.x) {

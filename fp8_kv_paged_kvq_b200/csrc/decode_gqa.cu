@@ -209,11 +209,13 @@ __global__ void __launch_bounds__(NW * 32, (NT == 1 ? 2 : 1))
   int32_t* pre = reinterpret_cast<int32_t*>(smem + K::kOffPre);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();                                 // the combine may launch (it waits for us)
   if (threadIdx.x == 0) {
     for (int i = 0; i < K::kSlots; ++i) mbar_init(&full[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
+  pdl_wait();                                    // the previous kernel (validate) has finished
   block_prefix_units(p, pre, scratch);           // includes __syncthreads
   if (blockIdx.x == 0)
     for (int b = threadIdx.x; b <= p.B; b += blockDim.x) p.ws_pre[b] = pre[b];
@@ -603,6 +605,7 @@ constexpr int kMaxPieces = 64;        // partials per segment at most
 constexpr int kCombOutputs = 4096;    // outputs per block (heads_per_block * Dv) at most
 
 __global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const CombineParams p) {
+  pdl_wait();                                    // the decode kernel has finished
   const int32_t seg = blockIdx.x;
   const int32_t b = seg / p.Hkv, h = seg - b * p.Hkv;
   const int32_t h0 = blockIdx.y * p.heads_per_block;            // first head of this block
@@ -722,8 +725,8 @@ cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const
   cp.heads_per_block = hpb;
   if (Dv % 4 != 0) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(B * Hkv), static_cast<unsigned>((G + hpb - 1) / hpb));
-  if (B * Hkv > 0) lse_combine_kernel<<<grid, kCombThreads, 0, stream>>>(cp);
-  return cudaGetLastError();
+  if (B * Hkv == 0) return cudaSuccess;
+  return launch_pdl(lse_combine_kernel, grid, dim3(kCombThreads), 0, stream, cp);
 }
 
 // Opt the kernel into the largest dynamic shared memory it can ask for, once
@@ -770,8 +773,7 @@ static cudaError_t run_gqa(const DecodeArgs& a, const CUtensorMap& km, const CUt
   p.ws_pre = reinterpret_cast<int32_t*>(ws + wl.off_pre);
   p.ws_lse = reinterpret_cast<float*>(ws + wl.off_lse);
   p.ws_o = reinterpret_cast<float*>(ws + wl.off_o);
-  kern<<<a.num_ctas, K::kThreads, smem, a.stream>>>(km, vm, p);
-  e = cudaGetLastError();
+  e = launch_pdl(kern, dim3(a.num_ctas), dim3(K::kThreads), smem, a.stream, km, vm, p);
   if (e != cudaSuccess) return e;
   return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, a.c.Hkv, p.G, a.Hq, a.c.Dv,
                             a.num_ctas, a.out, a.lse, a.stream);

@@ -168,6 +168,8 @@ __device__ __forceinline__ int32_t seq_tokens(const Params& p, int b) {
 // ceil(tokens_b / 64) into ws_pre[0..B].
 constexpr int kPrepThreads = 256;
 __global__ void __launch_bounds__(kPrepThreads) wide_prep_kernel(const Params p) {
+  pdl_trigger();                                 // the decode kernel may launch and set up
+  pdl_wait();                                    // the previous kernel (validate) has finished
   const int tid = threadIdx.x;
   if (blockIdx.x == 2 * p.B) {
     __shared__ int32_t scratch[kPrepThreads];
@@ -365,6 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *tmem_slot;
   const int pair = blockIdx.x >> 1;
   cluster_sync_all();                            // both CTAs' barriers and TMEM ready
+  pdl_trigger();                                 // the combine may launch (it waits for us)
+  pdl_wait();                                    // the pre-pass has finished
 
   const int64_t U = __ldg(p.ws_pre + p.B);
   const int32_t u0 = static_cast<int32_t>(U * pair / p.num_pairs);
@@ -848,21 +852,23 @@ cudaError_t launch_wide_decode(const DecodeArgs& a, const CUtensorMap& kqk,
   p.ws_lse = reinterpret_cast<float*>(ws + wl.off_lse);
   p.ws_o = reinterpret_cast<float*>(ws + wl.off_o);
   p.ws_q = ws + wl.off_extra;
-  wide::wide_prep_kernel<<<2 * a.B + 1, wide::kPrepThreads, 0, a.stream>>>(p);
-  e = cudaGetLastError();
+  e = launch_pdl(wide::wide_prep_kernel, dim3(2 * a.B + 1), dim3(wide::kPrepThreads), 0,
+                 a.stream, p);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * a.num_ctas);
   cfg.blockDim = dim3(wide::kThreads);
   cfg.dynamicSmemBytes = wide::kSmemBytes;
   cfg.stream = a.stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, wide::wide_decode_kernel, kqk, ktail, p);
   if (e != cudaSuccess) return e;
   return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, 1, wide::kHq, wide::kHq, wide::kDv,

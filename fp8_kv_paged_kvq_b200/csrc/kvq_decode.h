@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -46,6 +48,25 @@ inline WorkspaceLayout workspace_layout(int32_t B, int32_t Hkv, int32_t G, int32
   w.off_extra = align_up(w.off_o + slots * G * static_cast<size_t>(Dv) * 4, 256);
   w.total = align_up(w.off_extra + static_cast<size_t>(B) * extra_per_seq, 256);
   return w;
+}
+
+// Launch a kernel as a programmatic dependent of the previous kernel in the
+// stream: it may start launching early, and waits (griddepcontrol.wait)
+// before reading that kernel's results.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 int gqa_default_ctas(bool fp8, int D, int G, int B);

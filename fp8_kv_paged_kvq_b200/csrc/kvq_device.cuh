@@ -23,6 +23,16 @@ constexpr float kLn2 = 0.6931471805599453f;
 // ---------------------------------------------------------------------------
 // Timers, shared-memory addresses
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  pdl_trigger lets the next kernel of the
+// stream start launching once every CTA of this grid has called it (or
+// exited); pdl_wait, in that next kernel, returns once this grid has
+// completed and its writes are visible.  Both are no-ops for kernels not
+// launched with programmatic stream serialization.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -31,6 +31,11 @@ __global__ void __launch_bounds__(kValThreads)
                     const int32_t* __restrict__ block_table,
                     const uint32_t* __restrict__ expected, const int32_t* __restrict__ seq_lens,
                     int32_t ps, int32_t max_pages, uint8_t* __restrict__ abort_mask) {
+  // Launched as a programmatic dependent of the previous kernel (kvq_append
+  // in a decode step): the launch overlaps that kernel, and every global
+  // read here comes after it has finished.
+  pdl_trigger();
+  pdl_wait();
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
@@ -90,13 +95,15 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
   cfg.gridDim = dim3(static_cast<unsigned>(B * C));
   cfg.blockDim = dim3(kValThreads);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, validate_kernel, tags, P, block_table, expected, seq_lens, ps,
                             max_pages, abort_mask);
 }

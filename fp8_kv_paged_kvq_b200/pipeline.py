@@ -117,31 +117,37 @@ class DecodeLoop:
         self.graphs = {}
 
     def _path(self, check_tags: bool, stream=None, ev=None):
+        """One step.  ev: None, [start, end], or [start, before validate,
+        before decode, end] (events between kernels also break the kernels'
+        programmatic launch overlap, so the two-event form times the step)."""
         db = self.batch
         st = torch.cuda.current_stream() if stream is None else stream
+        inner = ev is not None and len(ev) == 4
         if ev is not None:
             ev[0].record(st)
         append(db.cache, db.k_new, db.v_new, db.new_slots, self.realloc, stream)
-        if ev is not None:
+        if inner:
             ev[1].record(st)
         if check_tags:
             db.validate(stream)
-        if ev is not None:
+        if inner:
             ev[2].record(st)
         db.decode(use_abort=check_tags, stream=stream)
         if ev is not None:
-            ev[3].record(st)
+            ev[-1].record(st)
 
     def capture(self, stream) -> None:
-        """Capture the step's hot path, with and without the tag check, with timing
-        events between append, validate and decode recorded inside the graph."""
+        """Capture the step's hot path, with and without the tag check, each
+        twice: with timing events only around the step, and with events
+        between append, validate and decode as well."""
         for chk in (True, False):
             self._path(chk, stream)          # warm up outside capture
-            ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                self._path(chk, stream, ev)
-            self.graphs[chk] = (g, ev)
+            for n_ev in (2, 4):
+                ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    self._path(chk, stream, ev)
+                self.graphs[(chk, n_ev == 4)] = (g, ev)
 
     def _flat(self, entries):
         return torch.tensor([b * self.cap + i for b, i in entries], dtype=torch.long,
@@ -181,10 +187,11 @@ class DecodeLoop:
         if stale_idx is not None:
             self.batch.expected.view(-1)[stale_idx] ^= 1
 
-    def run(self, check_tags: bool, stream):
-        """Replay the step's graph.  Returns its four events (before append, before
-        validate, before decode, after decode); they are reused by the next replay of
-        the same graph, so read them after synchronizing and before replaying again."""
-        g, ev = self.graphs[check_tags]
+    def run(self, check_tags: bool, stream, detailed: bool = False):
+        """Replay the step's graph.  Returns its events: (start, end), or with
+        detailed=True (before append, before validate, before decode, after
+        decode); they are reused by the next replay of the same graph, so read
+        them after synchronizing and before replaying again."""
+        g, ev = self.graphs[(check_tags, detailed)]
         g.replay()
         return ev
