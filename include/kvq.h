@@ -194,7 +194,14 @@ size_t kvq_decode_workspace_size(const kvq_cache* cache, int32_t B, int32_t num_
  * Requires cache->dtype == KVQ_FP8_E4M3.  Supported shapes: Dk == Dv in
  * {64, 128} with separate V pages, ps a multiple of 16 and
  * num_q_heads / Hkv <= 16; or Dk = 576, Dv = 512 with V aliasing K, one KV
- * head, 128 query heads, TOKEN scales and ps a multiple of 64.
+ * head, 128 query heads, TOKEN scales and ps a multiple of 64.  The second
+ * shape runs on the tensor cores: each query row is scaled by a power of
+ * two to a maximum in [128, 256) and split into two E4M3 terms (any BF16
+ * range; exact for scaled elements of magnitude >= 2^-2, smaller ones are
+ * rounded at the E4M3 step 2^-9), and the E4M3 NaN
+ * codes 0x7F / 0xFF, which kvq_append never writes, read as +-480 there.
+ * The kernels are launched as programmatic dependents of the previous work
+ * on the stream and wait for it before reading any argument.
  */
 kvq_status kvq_decode(const kvq_cache* cache, const void* q, int32_t num_q_heads,
                       const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
