@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--loop-steps", type=int, default=1000,
                     help="decode steps of the long workload's loop")
+    ap.add_argument("--sweep", action="store_true",
+                    help="capacity and concurrency sweep (FP8 vs BF16 at B = 1..64) instead of the bench line")
     ap.add_argument("--seqs", type=int, default=0,
                     help="keep only the first N sequences (smaller case for profiling)")
     return ap.parse_args()
@@ -461,6 +463,8 @@ def run_ours(args):
     if bf16:
         line["bf16_same_shape"] = bf16
         line["fp8_vs_bf16_step_time"] = ms_step / bf16["ms_per_step"]
+    if not is_wide(s) and s.kv_dtype == W.FP8 and not args.seqs:
+        line["bulk_append"] = run_bulk_append(s, dev, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=10.0)
     if rank == 0:
@@ -646,10 +650,97 @@ def run_bf16(wl_fp8, args, stream, world, dev):
     return res
 
 
+def run_bulk_append(spec, dev, stream, tokens=65536, iters=20):
+    """Bulk quantize: a prompt's worth of BF16 K/V (tokens x Hkv x D) through
+    kvq_append into FP8 pages scattered by a random page permutation, as at
+    the prefill -> decode hand-over.  Algorithmic bytes: the BF16 reads, the
+    code writes and the slot mapping."""
+    import fp8_kv_paged_kvq_b200 as kvq
+    s = spec
+    ps, H, Dk, Dv = s.page_size, s.num_kv_heads, s.head_dim_k, s.head_dim_v
+    pages = -(-tokens // ps)
+    g = torch.Generator(device=dev).manual_seed(11)
+    cache = kvq.PagedCache(kvq.FP8_E4M3, kvq.SCALE_HEAD, pages, ps, H, Dk, Dv, device=dev)
+    cache.k_scale.fill_(1.0 / 64)
+    cache.v_scale.fill_(1.0 / 64)
+    k = torch.randn(tokens, H, Dk, device=dev, generator=g).to(torch.bfloat16)
+    v = torch.randn(tokens, H, Dv, device=dev, generator=g).to(torch.bfloat16)
+    perm = torch.randperm(pages, device=dev, generator=g).to(torch.int32)
+    t = torch.arange(tokens, device=dev, dtype=torch.int32)
+    slots = (perm[t // ps] * ps + t % ps).contiguous()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            kvq.append(cache, k, v, slots, stream=stream)
+        gr = capture(lambda: kvq.append(cache, k, v, slots, stream=stream), stream)
+        ms = time_graph(gr, iters, stream)
+    nbytes = tokens * H * (Dk + Dv) * 3 + tokens * 4
+    hbm, kind = peaks()
+    del gr
+    return {"tokens": tokens, "ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+            "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm, "peak_kind": kind,
+            "bytes": nbytes, "note": "bf16 K/V read + e4m3 codes written + slot mapping"}
+
+
+def run_sweep(args):
+    """Capacity and concurrency sweep on the gqa shape (64 query / 8 KV heads,
+    d 128, page 16, 8,192 tokens per sequence): FP8 and BF16 decode time at
+    B = 1, 8, 16, 32, 64, and the tokens a fixed memory budget holds in each
+    format (cache bytes per token read from the allocated pages)."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    import fp8_kv_paged_kvq_b200 as kvq
+    from fp8_kv_paged_kvq_b200 import build as kvq_build
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch
+    kvq_build.build()
+    stream = torch.cuda.Stream(device=dev)
+    hbm, _ = peaks()
+    rows = []
+    budget = 80 * 2**30                       # bytes of cache in the capacity comparison
+    per_token = {}
+    for B in (1, 8, 16, 32, 64):
+        row = {"B": B}
+        for dt in (W.FP8, W.BF16):
+            spec = W.spec_by_name("gqa")
+            spec.seq_lens = [8192] * B
+            spec.kv_dtype = dt
+            wl = W.make_workload(spec, seed=0, device=dev)
+            db = DecodeBatch(wl, device=dev)
+            db.prefill()
+            c = db.cache
+            nbytes = sum(x.numel() * x.element_size() for x in
+                         (c.k_pages, c.v_pages, c.k_scale, c.v_scale) if x is not None)
+            per_token[dt] = nbytes / (wl.num_pages * spec.page_size)
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    db.decode(use_abort=False, stream=stream)
+                gd = capture(lambda: db.decode(use_abort=False, stream=stream), stream)
+                ms = time_graph(gd, args.steps, stream)
+            kv = wl.kv_bytes_read()               # bytes of this cache format
+            row[dt] = {"ms": ms, "kv_gbs": kv / (ms * 1e-3) / 1e9,
+                       "frac_of_hbm": kv / (ms * 1e-3) / 1e9 / hbm,
+                       "decode_tokens_per_s": B / (ms * 1e-3)}
+            del gd, db
+            torch.cuda.empty_cache()
+        row["fp8_over_bf16_time"] = row[W.FP8]["ms"] / row[W.BF16]["ms"]
+        rows.append(row)
+    line = {"sweep": "gqa shape, 8,192 tokens per sequence, decode call only",
+            "rows": rows,
+            "capacity": {"budget_bytes": budget,
+                         "fp8_bytes_per_token": per_token[W.FP8],
+                         "bf16_bytes_per_token": per_token[W.BF16],
+                         "fp8_tokens": int(budget // per_token[W.FP8]),
+                         "bf16_tokens": int(budget // per_token[W.BF16])},
+            "steps": args.steps}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     elif args.workload == "long":
         run_long(args)
     else:

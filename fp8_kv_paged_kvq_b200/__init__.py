@@ -65,7 +65,7 @@ def lib() -> ctypes.CDLL:
         L.kvq_amax.argtypes = [_VP, _I64, _I32, _I32, _I32, _VP, _VP]
         L.kvq_scale_from_amax.argtypes = [_VP, _VP, _I32, _VP]
         L.kvq_append.argtypes = [ctypes.POINTER(KvqCacheDesc), _VP, _VP, _VP, _I32, _VP, _I32, _VP]
-        L.kvq_validate.argtypes = [_VP, _I32, _VP, _VP, _VP, _I32, _I32, _I32, _VP, _VP]
+        L.kvq_validate.argtypes = [_VP, _I32, _VP, _VP, _VP, _I32, _I32, _I32, _VP, _VP, _VP, _VP]
         L.kvq_decode_workspace_size.restype = ctypes.c_size_t
         L.kvq_decode_workspace_size.argtypes = [ctypes.POINTER(KvqCacheDesc), _I32, _I32, _I32]
         dec = [ctypes.POINTER(KvqCacheDesc), _VP, _I32, _VP, _I32, _VP, _I32, _VP, ctypes.c_float,
@@ -75,9 +75,11 @@ def lib() -> ctypes.CDLL:
         L.kvq_decode_noalloc.argtypes = [ctypes.POINTER(KvqCacheDesc), _VP, _I32, _VP, _I32, _VP,
                                          _I32, _VP, ctypes.c_float, _VP, _VP, _I32, _VP]
         L.kvq_e4m3_encode_bits.argtypes = [_U32, _U32, _VP, _VP]
+        L.kvq_e4m3_quantize_bits.argtypes = [_U32, _U32, ctypes.c_float, _VP, _VP]
         L.kvq_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
         for f in ("kvq_amax", "kvq_scale_from_amax", "kvq_append", "kvq_validate", "kvq_decode",
                   "kvq_decode_bf16", "kvq_decode_noalloc", "kvq_e4m3_encode_bits",
+                  "kvq_e4m3_quantize_bits",
                   "kvq_device_error"):
             getattr(L, f).restype = _I32
         _lib = L
@@ -191,13 +193,18 @@ def append(cache: PagedCache, k_new: torch.Tensor, v_new: Optional[torch.Tensor]
 
 def validate(page_tags: torch.Tensor, block_table: torch.Tensor, expected_tags: torch.Tensor,
              seq_lens: torch.Tensor, page_size: int, abort_mask: Optional[torch.Tensor] = None,
-             stream=None) -> torch.Tensor:
+             stream=None, n_aborted: Optional[torch.Tensor] = None,
+             first_bad: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Abort mask u8 [B].  Optional telemetry, filled on the device: n_aborted
+    (int32 [1]) = aborted requests; first_bad (int32 [B]) = each request's
+    first failing block-table index, or -1."""
     B, max_pages = block_table.shape
     if abort_mask is None:
         abort_mask = torch.empty(B, dtype=torch.uint8, device=block_table.device)
     _check("kvq_validate", lib().kvq_validate(
         _ptr(page_tags), page_tags.numel(), _ptr(block_table), _ptr(expected_tags),
-        _ptr(seq_lens), page_size, B, max_pages, _ptr(abort_mask), _stream(stream)))
+        _ptr(seq_lens), page_size, B, max_pages, _ptr(abort_mask), _ptr(n_aborted),
+        _ptr(first_bad), _stream(stream)))
     return abort_mask
 
 
@@ -255,6 +262,17 @@ def e4m3_encode_bits(start: int, count: int, out: Optional[torch.Tensor] = None,
         out = torch.empty(count, dtype=torch.uint8, device="cuda")
     _check("kvq_e4m3_encode_bits",
            lib().kvq_e4m3_encode_bits(start, count, _ptr(out), _stream(stream)))
+    return out
+
+
+def e4m3_quantize_bits(start: int, count: int, scale: float,
+                       out: Optional[torch.Tensor] = None, stream=None):
+    """E4M3 codes of (float with bit pattern start + i) / scale, as kvq_append divides."""
+    if out is None:
+        out = torch.empty(count, dtype=torch.uint8, device="cuda")
+    _check("kvq_e4m3_quantize_bits",
+           lib().kvq_e4m3_quantize_bits(start, count, ctypes.c_float(scale), _ptr(out),
+                                        _stream(stream)))
     return out
 
 

@@ -245,14 +245,13 @@ kvq_status kvq_append(const kvq_cache* cache, const void* k_new, const void* v_n
 kvq_status kvq_validate(const uint32_t* page_tags, int32_t num_pages, const int32_t* block_table,
                         const uint32_t* expected_tags, const int32_t* seq_lens,
                         int32_t page_size, int32_t B, int32_t max_pages, uint8_t* abort_mask,
-                        void* stream) {
+                        int32_t* n_aborted, int32_t* first_bad, void* stream) {
   if (num_pages < 1 || page_size < 1 || B < 0 || max_pages < 1) return KVQ_ERR_INVALID_ARG;
-  if (B == 0) return KVQ_OK;
-  if (page_tags == nullptr || block_table == nullptr || expected_tags == nullptr ||
-      seq_lens == nullptr || abort_mask == nullptr)
+  if (B > 0 && (page_tags == nullptr || block_table == nullptr || expected_tags == nullptr ||
+                seq_lens == nullptr || abort_mask == nullptr))
     return KVQ_ERR_INVALID_ARG;
   return from_cuda(launch_validate(page_tags, num_pages, block_table, expected_tags, seq_lens,
-                                   page_size, B, max_pages, abort_mask,
+                                   page_size, B, max_pages, abort_mask, n_aborted, first_bad,
                                    static_cast<cudaStream_t>(stream)));
 }
 
@@ -288,6 +287,12 @@ kvq_status kvq_decode_bf16(const kvq_cache* cache, const void* q, int32_t num_q_
   return decode_common(false, cache, q, num_q_heads, block_table, max_pages, seq_lens, B,
                        abort_mask, sm_scale, out, lse, workspace, workspace_bytes, num_ctas,
                        stream);
+}
+
+kvq_status kvq_e4m3_quantize_bits(uint32_t start, uint32_t count, float scale, uint8_t* out,
+                                  void* stream) {
+  if (out == nullptr || !(scale > 0.0f) || scale == __builtin_inff()) return KVQ_ERR_INVALID_ARG;
+  return from_cuda(launch_quantize_bits(start, count, scale, out, static_cast<cudaStream_t>(stream)));
 }
 
 kvq_status kvq_e4m3_encode_bits(uint32_t start, uint32_t count, uint8_t* out, void* stream) {

@@ -61,53 +61,33 @@ __global__ void scale_from_amax_kernel(const float* __restrict__ amax, float* __
 
 // ---------------------------------------------------------------------------
 // Append: one warp per (token, kv head); the last block also bumps tags.
+// The warp's lanes take the row's 8-value groups in turn across the K row
+// and then the V row (for head dims 128 that is one group per lane), so a
+// half-warp writes 128 contiguous code bytes with 8-byte stores.
 // ---------------------------------------------------------------------------
-// Quantize one row of D bf16 values (D % 16 == 0) into E4M3 codes at dst
-// with 16-byte stores; s is the row's scale.
-__device__ __forceinline__ void quantize_row(const uint16_t* __restrict__ src,
-                                             uint8_t* __restrict__ dst, int32_t D, float s,
-                                             int lane) {
-  for (int32_t g = lane; g < D / 16; g += 32) {
-    const uint4 a = *reinterpret_cast<const uint4*>(src + g * 16);
-    const uint4 b = *reinterpret_cast<const uint4*>(src + g * 16 + 8);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t pairs[8];
+// Eight bf16 values to eight E4M3 codes of v / s (IEEE binary32 division,
+// then rounding to nearest even with saturation in the conversion).
+__device__ __forceinline__ uint2 quantize8(const uint4 a, float s) {
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+  uint32_t pairs[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float lo = __fdiv_rn(bf16lo_to_f32(w[k]), s);
-      const float hi = __fdiv_rn(bf16hi_to_f32(w[k]), s);
-      pairs[k] = f32x2_to_e4m3x2(lo, hi);               // 16 bits: lo code | hi code << 8
-    }
-    uint4 out;
-    out.x = pairs[0] | (pairs[1] << 16);
-    out.y = pairs[2] | (pairs[3] << 16);
-    out.z = pairs[4] | (pairs[5] << 16);
-    out.w = pairs[6] | (pairs[7] << 16);
-    *reinterpret_cast<uint4*>(dst + g * 16) = out;
-  }
+  for (int k = 0; k < 4; ++k)
+    pairs[k] = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[k]), s),
+                               __fdiv_rn(bf16hi_to_f32(w[k]), s));   // lo code | hi code << 8
+  return make_uint2(pairs[0] | (pairs[1] << 16), pairs[2] | (pairs[3] << 16));
 }
 
-__device__ __forceinline__ float row_amax(const uint16_t* __restrict__ src, int32_t D, int lane) {
+__device__ __forceinline__ float amax8(const uint4 a) {
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
   float m = 0.0f;
-  for (int32_t g = lane; g < D / 8; g += 32) {
-    const uint4 a = *reinterpret_cast<const uint4*>(src + g * 8);
-    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      m = fmaxf(m, fabsf(bf16lo_to_f32(w[k])));
-      m = fmaxf(m, fabsf(bf16hi_to_f32(w[k])));
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  return m;
+  for (int k = 0; k < 4; ++k)
+    m = fmaxf(m, fmaxf(fabsf(bf16lo_to_f32(w[k])), fabsf(bf16hi_to_f32(w[k]))));
+  return m;                                   // fmaxf drops NaN operands
 }
 
-__device__ __forceinline__ void copy_row_bf16(const uint16_t* __restrict__ src,
-                                              uint16_t* __restrict__ dst, int32_t D, int lane) {
-  for (int32_t g = lane; g < D / 8; g += 32)
-    *reinterpret_cast<uint4*>(dst + g * 8) = *reinterpret_cast<const uint4*>(src + g * 8);
-}
+constexpr int kAppendWarps = 8;
+constexpr int kRowsPerWarp = 4;      // (token, head) rows per warp in the batched case
 
 struct AppendArgs {
   CacheView c;
@@ -118,9 +98,61 @@ struct AppendArgs {
   const int32_t* realloc_pages;
   int32_t n_realloc;
   int32_t token_blocks;  // blocks that handle tokens; the next block bumps tags
+  int32_t batched;       // rows per warp: kRowsPerWarp (batched case) or 1
 };
 
-constexpr int kAppendWarps = 8;
+// The common case: K and V rows of at most 32 eight-value groups together
+// (head dims up to 128) with a per-tensor or per-head scale.  A warp takes
+// kRowsPerWarp rows and issues all their loads before converting any, so
+// four 16-byte loads per lane are in flight.  Rows run token-major within a
+// head (row r: head r / T, token r % T), so a warp writes consecutive slots
+// of one head: contiguous bytes when the tokens' slots are consecutive.
+template <bool FP8>
+__device__ __forceinline__ void append_rows_batched(const AppendArgs& a, int64_t row0, int lane) {
+  const CacheView& c = a.c;
+  const int64_t rows = static_cast<int64_t>(a.T) * c.Hkv;
+  const int32_t nk = c.Dk / 8, nv = c.Dv / 8;
+  const bool isk = lane < nk, active = lane < nk + nv;
+  const int32_t e = 8 * (isk ? lane : lane - nk);
+  uint4 x[kRowsPerWarp];
+  int64_t prow[kRowsPerWarp];
+  int32_t hh[kRowsPerWarp];
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    const int64_t r = row0 + i;
+    prow[i] = -1;
+    hh[i] = 0;
+    x[i] = make_uint4(0, 0, 0, 0);
+    if (r < rows) {
+      const int32_t h = static_cast<int32_t>(r / a.T), t = static_cast<int32_t>(r % a.T);
+      const int64_t slot = a.slot_mapping[t];
+      hh[i] = h;
+      if (slot >= 0 && slot < static_cast<int64_t>(c.P) * c.ps)
+        prow[i] = ((slot / c.ps) * c.Hkv + h) * c.ps + slot % c.ps;
+      if (active)
+        x[i] = __ldg(reinterpret_cast<const uint4*>(
+            (isk ? a.k_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dk
+                 : a.v_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dv) + e));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    if (prow[i] < 0 || !active) continue;
+    if (FP8) {
+      const float* sc = isk ? c.k_scale : c.v_scale;
+      const float s = sc[c.scale_mode == 0 ? 0 : hh[i]];
+      uint8_t* dst = static_cast<uint8_t*>(isk ? c.k_pages : c.v_pages) +
+                     prow[i] * (isk ? c.Dk : c.Dv) + e;
+      *reinterpret_cast<uint2*>(dst) = quantize8(x[i], s);
+    } else {
+      uint16_t* dst = static_cast<uint16_t*>(isk ? c.k_pages : c.v_pages) +
+                      prow[i] * (isk ? c.Dk : c.Dv) + e;
+      *reinterpret_cast<uint4*>(dst) = x[i];
+    }
+  }
+}
+
+
 
 __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a) {
   pdl_trigger();            // the tag check may start loading its block-table entries
@@ -133,6 +165,13 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a)
     return;
   }
   const int lane = threadIdx.x & 31;
+  if (a.batched > 1) {
+    const int64_t row0 =
+        (static_cast<int64_t>(blockIdx.x) * kAppendWarps + (threadIdx.x >> 5)) * kRowsPerWarp;
+    if (c.fp8) append_rows_batched<true>(a, row0, lane);
+    else append_rows_batched<false>(a, row0, lane);
+    return;
+  }
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kAppendWarps + (threadIdx.x >> 5);
   if (row >= static_cast<int64_t>(a.T) * c.Hkv) return;
   const int32_t t = static_cast<int32_t>(row / c.Hkv);
@@ -141,28 +180,53 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a)
   if (slot < 0 || slot >= static_cast<int64_t>(c.P) * c.ps) return;
   const int64_t p = slot / c.ps, o = slot % c.ps;
   const int64_t prow = (p * c.Hkv + h) * c.ps + o;   // [P][Hkv][ps] row index
-  for (int part = 0; part < 2; ++part) {
-    if (part == 1 && c.v_pages == nullptr) break;
-    const int32_t D = part ? c.Dv : c.Dk;
-    const uint16_t* src = (part ? a.v_new : a.k_new) + (static_cast<int64_t>(t) * c.Hkv + h) * D;
-    if (!c.fp8) {
-      uint16_t* dst = static_cast<uint16_t*>(part ? c.v_pages : c.k_pages) + prow * D;
-      copy_row_bf16(src, dst, D, lane);
-      continue;
+  const int32_t nk = c.Dk / 8, nv = c.v_pages == nullptr ? 0 : c.Dv / 8;
+  const uint16_t* ksrc = a.k_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dk;
+  const uint16_t* vsrc = a.v_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dv;
+  if (!c.fp8) {
+    uint16_t* kdst = static_cast<uint16_t*>(c.k_pages) + prow * c.Dk;
+    uint16_t* vdst = static_cast<uint16_t*>(c.v_pages) + prow * c.Dv;
+    for (int32_t g = lane; g < nk + nv; g += 32) {
+      const bool isk = g < nk;
+      const int32_t e = 8 * (isk ? g : g - nk);
+      *reinterpret_cast<uint4*>((isk ? kdst : vdst) + e) =
+          *reinterpret_cast<const uint4*>((isk ? ksrc : vsrc) + e);
     }
-    float* sc = part ? c.v_scale : c.k_scale;
-    float s;
-    if (c.scale_mode == 0) {
-      s = sc[0];
-    } else if (c.scale_mode == 1) {
-      s = sc[h];
-    } else {
-      const float amax = row_amax(src, D, lane);
-      s = (amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
-      if (lane == 0) sc[prow] = s;
+    return;
+  }
+  float sk, sv = 1.0f;
+  if (c.scale_mode == 0) {
+    sk = c.k_scale[0];
+    if (nv) sv = c.v_scale[0];
+  } else if (c.scale_mode == 1) {
+    sk = c.k_scale[h];
+    if (nv) sv = c.v_scale[h];
+  } else {
+    // per-token scale: amax over each row, reduced across the warp
+    float ak = 0.0f, av = 0.0f;
+    for (int32_t g = lane; g < nk + nv; g += 32) {
+      if (g < nk) ak = fmaxf(ak, amax8(*reinterpret_cast<const uint4*>(ksrc + 8 * g)));
+      else av = fmaxf(av, amax8(*reinterpret_cast<const uint4*>(vsrc + 8 * (g - nk))));
     }
-    uint8_t* dst = static_cast<uint8_t*>(part ? c.v_pages : c.k_pages) + prow * D;
-    quantize_row(src, dst, D, s, lane);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, off));
+      av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, off));
+    }
+    sk = (ak > 0.0f) ? __fdiv_rn(ak, 448.0f) : 1.0f;
+    sv = (av > 0.0f) ? __fdiv_rn(av, 448.0f) : 1.0f;
+    if (lane == 0) {
+      c.k_scale[prow] = sk;
+      if (nv) c.v_scale[prow] = sv;
+    }
+  }
+  uint8_t* kdst = static_cast<uint8_t*>(c.k_pages) + prow * c.Dk;
+  uint8_t* vdst = nv ? static_cast<uint8_t*>(c.v_pages) + prow * c.Dv : nullptr;
+  for (int32_t g = lane; g < nk + nv; g += 32) {
+    const bool isk = g < nk;
+    const int32_t e = 8 * (isk ? g : g - nk);
+    const uint4 x = *reinterpret_cast<const uint4*>((isk ? ksrc : vsrc) + e);
+    *reinterpret_cast<uint2*>((isk ? kdst : vdst) + e) = quantize8(x, isk ? sk : sv);
   }
 }
 
@@ -218,10 +282,32 @@ cudaError_t launch_append(const CacheView& c, const uint16_t* k_new, const uint1
   a.realloc_pages = realloc_pages;
   a.n_realloc = n_realloc;
   const int64_t rows = static_cast<int64_t>(T) * c.Hkv;
-  a.token_blocks = static_cast<int32_t>((rows + kAppendWarps - 1) / kAppendWarps);
+  const bool batched = c.v_pages != nullptr && c.Dk / 8 + c.Dv / 8 <= 32 &&
+                       (!c.fp8 || c.scale_mode != 2);
+  a.batched = batched ? kRowsPerWarp : 1;
+  const int64_t per_block = static_cast<int64_t>(kAppendWarps) * a.batched;
+  a.token_blocks = static_cast<int32_t>((rows + per_block - 1) / per_block);
   const int32_t blocks = a.token_blocks + (n_realloc > 0 ? 1 : 0);
   if (blocks == 0) return cudaSuccess;
   append_kernel<<<blocks, kAppendWarps * 32, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// Exhaustive check of the append path's quantize step:
+// out[i] = E(bits(start + i) / scale) with the same division and conversion.
+__global__ void quantize_bits_kernel(uint32_t start, uint32_t count, float scale,
+                                     uint8_t* __restrict__ out) {
+  const uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= count) return;
+  const float q = __fdiv_rn(__uint_as_float(start + static_cast<uint32_t>(i)), scale);
+  out[i] = static_cast<uint8_t>(f32x2_to_e4m3x2(q, 0.0f) & 0xFFu);
+}
+
+cudaError_t launch_quantize_bits(uint32_t start, uint32_t count, float scale, uint8_t* out,
+                                 cudaStream_t stream) {
+  if (count == 0) return cudaSuccess;
+  quantize_bits_kernel<<<static_cast<unsigned>((static_cast<uint64_t>(count) + 255) / 256), 256,
+                         0, stream>>>(start, count, scale, out);
   return cudaGetLastError();
 }
 

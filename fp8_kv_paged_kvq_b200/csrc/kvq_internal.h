@@ -25,12 +25,14 @@ cudaError_t launch_scale_from_amax(const float* amax, float* scale, int32_t n,
 cudaError_t launch_append(const CacheView& c, const uint16_t* k_new, const uint16_t* v_new,
                           const int32_t* slot_mapping, int32_t T, const int32_t* realloc_pages,
                           int32_t n_realloc, cudaStream_t stream);
+cudaError_t launch_quantize_bits(uint32_t start, uint32_t count, float scale, uint8_t* out,
+                                 cudaStream_t stream);
 cudaError_t launch_encode_bits(uint32_t start, uint32_t count, uint8_t* out,
                                cudaStream_t stream);
 cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* block_table,
                             const uint32_t* expected, const int32_t* seq_lens, int32_t ps,
                             int32_t B, int32_t max_pages, uint8_t* abort_mask,
-                            cudaStream_t stream);
+                            int32_t* n_aborted, int32_t* first_bad, cudaStream_t stream);
 cudaError_t read_and_clear_error_flags(uint32_t* flags);
 
 }  // namespace kvq

@@ -30,7 +30,8 @@ __global__ void __launch_bounds__(kValThreads)
     validate_kernel(const uint32_t* __restrict__ tags, int32_t P,
                     const int32_t* __restrict__ block_table,
                     const uint32_t* __restrict__ expected, const int32_t* __restrict__ seq_lens,
-                    int32_t ps, int32_t max_pages, uint8_t* __restrict__ abort_mask) {
+                    int32_t ps, int32_t max_pages, uint8_t* __restrict__ abort_mask,
+                    int32_t* __restrict__ n_aborted, int32_t* __restrict__ first_bad) {
   // Launched as a programmatic dependent of the previous kernel (kvq_append
   // in a decode step): the launch overlaps that kernel, and every global
   // read here comes after it has finished.
@@ -40,7 +41,8 @@ __global__ void __launch_bounds__(kValThreads)
   const int C = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
   const int32_t b = blockIdx.x / C;
-  __shared__ int flag;
+  __shared__ int32_t flag;          // this CTA's first failing entry, or INT32_MAX
+  __shared__ int32_t warp_min[kValThreads / 32];
   int64_t n = seq_lens[b];
   n = n < 0 ? 0 : n;
   const int64_t cap = static_cast<int64_t>(max_pages) * ps;
@@ -48,7 +50,7 @@ __global__ void __launch_bounds__(kValThreads)
   const int32_t npages = static_cast<int32_t>((n + ps - 1) / ps);
   const int32_t* bt = block_table + static_cast<int64_t>(b) * max_pages;
   const uint32_t* ex = expected + static_cast<int64_t>(b) * max_pages;
-  int bad = 0;
+  int32_t bad = INT32_MAX;          // smallest failing block-table index seen
   for (int32_t base = rank * kPerCta; base < npages; base += C * kPerCta) {
     int32_t page[kPerThread];
     uint32_t want[kPerThread];
@@ -67,18 +69,26 @@ __global__ void __launch_bounds__(kValThreads)
       const int32_t i = base + k * kValThreads + threadIdx.x;
       if (i < npages) {
         const int32_t p = page[k];
-        if (p < 0 || p >= P) bad = 1;
-        else if (tags[p] != want[k]) bad = 1;
+        if (p < 0 || p >= P || tags[p] != want[k]) bad = min(bad, i);
       }
     }
   }
-  const int any = __syncthreads_or(bad);
-  if (threadIdx.x == 0) flag = any;
+  bad = __reduce_min_sync(0xffffffffu, bad);
+  if ((threadIdx.x & 31) == 0) warp_min[threadIdx.x >> 5] = bad;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t m = INT32_MAX;
+    for (int w = 0; w < kValThreads / 32; ++w) m = min(m, warp_min[w]);
+    flag = m;
+  }
   cluster.sync();
   if (rank == 0 && threadIdx.x == 0) {
-    int all = 0;
-    for (int r = 0; r < C; ++r) all |= *cluster.map_shared_rank(&flag, r);
-    abort_mask[b] = all ? 1 : 0;
+    int32_t first = INT32_MAX;
+    for (int r = 0; r < C; ++r) first = min(first, *cluster.map_shared_rank(&flag, r));
+    const bool aborted = first != INT32_MAX;
+    abort_mask[b] = aborted ? 1 : 0;
+    if (first_bad != nullptr) first_bad[b] = aborted ? first : -1;
+    if (n_aborted != nullptr && aborted) atomicAdd(n_aborted, 1);
   }
   cluster.sync();   // every CTA's flag stays alive until rank 0 has read it
 }
@@ -86,7 +96,11 @@ __global__ void __launch_bounds__(kValThreads)
 cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* block_table,
                             const uint32_t* expected, const int32_t* seq_lens, int32_t ps,
                             int32_t B, int32_t max_pages, uint8_t* abort_mask,
-                            cudaStream_t stream) {
+                            int32_t* n_aborted, int32_t* first_bad, cudaStream_t stream) {
+  if (n_aborted != nullptr) {
+    const cudaError_t e = cudaMemsetAsync(n_aborted, 0, sizeof(int32_t), stream);
+    if (e != cudaSuccess) return e;
+  }
   if (B == 0) return cudaSuccess;
   int C = (max_pages + kPerCta - 1) / kPerCta;
   C = C < 1 ? 1 : (C > kMaxCluster ? kMaxCluster : C);
@@ -105,7 +119,7 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, validate_kernel, tags, P, block_table, expected, seq_lens, ps,
-                            max_pages, abort_mask);
+                            max_pages, abort_mask, n_aborted, first_bad);
 }
 
 cudaError_t read_and_clear_error_flags(uint32_t* flags) {

@@ -150,13 +150,22 @@ kvq_status kvq_append(const kvq_cache* cache, const void* k_new, const void* v_n
  *   block_table[b][i] outside [0, num_pages) or
  *   page_tags[block_table[b][i]] != expected_tags[b][i],
  * else 0.  Entries of block_table / expected_tags beyond ceil(n/ps) are not
- * read.  One thread-block cluster of up to 8 CTAs checks each request.  block_table: i32 [B][max_pages]; expected_tags: u32 [B][max_pages];
- * seq_lens: i32 [B]; abort_mask: u8 [B] (written).
+ * read.  One thread-block cluster of up to 8 CTAs checks each request.
+ *   block_table i32 [B][max_pages]; expected_tags u32 [B][max_pages];
+ *   seq_lens i32 [B]; abort_mask u8 [B] (written).
+ * Optional telemetry (device pointers, NULL to skip), because the pages name
+ * the mismatch rate as the quantity to watch ([remio] "Sicherheit
+ * gemeinsamer KV-Caches wird zum Produktionsthema"):
+ *   n_aborted   i32 [1]: set to the number of aborted requests (zeroed on
+ *               the stream first, so it needs no initialisation);
+ *   first_bad   i32 [B]: the smallest failing index i of each request, or -1.
+ * Launched as a programmatic dependent of the previous kernel on the stream;
+ * it reads nothing before that kernel has finished.
  */
 kvq_status kvq_validate(const uint32_t* page_tags, int32_t num_pages, const int32_t* block_table,
                         const uint32_t* expected_tags, const int32_t* seq_lens,
                         int32_t page_size, int32_t B, int32_t max_pages, uint8_t* abort_mask,
-                        void* stream);
+                        int32_t* n_aborted, int32_t* first_bad, void* stream);
 
 /*
  * Bytes of device workspace kvq_decode / kvq_decode_bf16 need for this
@@ -250,6 +259,15 @@ kvq_status kvq_decode_noalloc(const kvq_cache* cache, const void* q, int32_t num
  * wrap mod 2^32).  out: u8 [count].
  */
 kvq_status kvq_e4m3_encode_bits(uint32_t start, uint32_t count, uint8_t* out, void* stream);
+
+/*
+ * The division kvq_append performs, exposed for exhaustive checks:
+ * out[i] = E4M3(x / scale) for x the float with bit pattern start + i,
+ * where x / scale is the IEEE binary32 quotient (round to nearest even).
+ * scale must be positive and finite.  out: u8 [count].
+ */
+kvq_status kvq_e4m3_quantize_bits(uint32_t start, uint32_t count, float scale, uint8_t* out,
+                                  void* stream);
 
 /*
  * Reads and clears the library's device-side error word on the current

@@ -80,6 +80,14 @@ def e4m3_encode_bits_range(start: int, count: int) -> np.ndarray:
     return out
 
 
+def e4m3_quantize_bits_range(start: int, count: int, scale: float) -> np.ndarray:
+    """Codes of (float bits start + i) / scale with IEEE binary32 division."""
+    out = np.empty(count, dtype=np.uint8)
+    lib().oracle_e4m3_quantize_bits_range(ctypes.c_uint32(start), ctypes.c_uint32(count),
+                                          ctypes.c_float(scale), _p(out))
+    return out
+
+
 def scale_from_amax(amax: float) -> float:
     return float(lib().oracle_scale_from_amax(ctypes.c_float(amax)))
 
@@ -141,17 +149,20 @@ def append(cache: Cache, k_new, v_new, slot_mapping, realloc_pages=None) -> None
                         ctypes.c_int32(0 if rp is None else rp.size))
 
 
-def validate(page_tags, block_table, expected_tags, seq_lens, page_size) -> np.ndarray:
+def validate(page_tags, block_table, expected_tags, seq_lens, page_size, first_bad=False):
+    """Abort mask u8 [B]; with first_bad=True also each request's first failing
+    block-table index (int32 [B], -1 if none)."""
     page_tags = np.ascontiguousarray(page_tags, dtype=np.uint32)
     block_table = np.ascontiguousarray(block_table, dtype=np.int32)
     expected_tags = np.ascontiguousarray(expected_tags, dtype=np.uint32)
     seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
     B, max_pages = block_table.shape
     out = np.empty(B, dtype=np.uint8)
+    fb = np.empty(B, dtype=np.int32) if first_bad else None
     lib().oracle_validate(_p(page_tags), ctypes.c_int32(page_tags.size), _p(block_table),
                           _p(expected_tags), _p(seq_lens), ctypes.c_int32(page_size),
-                          ctypes.c_int32(B), ctypes.c_int32(max_pages), _p(out))
-    return out
+                          ctypes.c_int32(B), ctypes.c_int32(max_pages), _p(out), _p(fb))
+    return (out, fb) if first_bad else out
 
 
 def decode(cache: Cache, q_bf16_bits, block_table, seq_lens, abort_mask, sm_scale, rows=None):

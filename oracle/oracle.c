@@ -134,6 +134,15 @@ void oracle_e4m3_encode_bits_range(uint32_t start, uint32_t count, uint8_t* out)
     out[i] = oracle_e4m3_encode(bits_to_float(start + (uint32_t)i));
 }
 
+/* Codes of (float with bit pattern start + i) / scale, the quotient being
+ * the IEEE binary32 division (this file is built without contraction or
+ * fast math): the quantize step of the append, R3. */
+void oracle_e4m3_quantize_bits_range(uint32_t start, uint32_t count, float scale, uint8_t* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < (int64_t)count; i++)
+    out[i] = oracle_e4m3_encode(bits_to_float(start + (uint32_t)i) / scale);
+}
+
 void oracle_e4m3_decode_array(const uint8_t* c, double* out, int64_t n) {
   for (int64_t i = 0; i < n; i++) out[i] = oracle_e4m3_decode(c[i]);
 }
@@ -260,16 +269,21 @@ static int64_t clamp_tokens(int32_t seq_len, int32_t max_pages, int32_t ps) {
  */
 void oracle_validate(const uint32_t* tags, int32_t P, const int32_t* block_table,
                      const uint32_t* expected, const int32_t* seq_lens, int32_t ps, int32_t B,
-                     int32_t max_pages, uint8_t* abort_mask) {
+                     int32_t max_pages, uint8_t* abort_mask, int32_t* first_bad) {
   for (int32_t b = 0; b < B; b++) {
     int64_t n = clamp_tokens(seq_lens[b], max_pages, ps);
     int64_t npages = (n + ps - 1) / ps;
     uint8_t bad = 0;
+    int32_t first = -1;   /* telemetry: the first entry that fails, in index order */
     for (int64_t i = 0; i < npages; i++) {
       int32_t p = block_table[(int64_t)b * max_pages + i];
-      if (p < 0 || p >= P || tags[p] != expected[(int64_t)b * max_pages + i]) bad = 1;
+      if (p < 0 || p >= P || tags[p] != expected[(int64_t)b * max_pages + i]) {
+        if (!bad) first = (int32_t)i;
+        bad = 1;
+      }
     }
     abort_mask[b] = bad;
+    if (first_bad) first_bad[b] = first;
   }
 }
 

@@ -48,8 +48,9 @@ def test_status_strings(lib):
 def test_host_checks_reject_bad_arguments_without_a_device(lib):
     E = kvq.KVQ_ERR_INVALID_ARG
     assert lib.kvq_append(None, None, None, None, 0, None, 0, None) == E
-    assert lib.kvq_validate(None, 1, None, None, None, 16, -1, 1, None, None) == E
-    assert lib.kvq_validate(None, 0, None, None, None, 16, 1, 1, None, None) == E
+    assert lib.kvq_validate(None, 1, None, None, None, 16, -1, 1, None, None, None, None) == E
+    assert lib.kvq_validate(None, 0, None, None, None, 16, 1, 1, None, None, None, None) == E
+    assert lib.kvq_validate(None, 4, None, None, None, 16, 1, 1, None, None, None, None) == E
     assert lib.kvq_amax(None, 4, 1, 12, 0, None, None) == E           # D % 8 != 0, null out
     assert lib.kvq_scale_from_amax(None, None, -1, None) == E
     assert lib.kvq_e4m3_encode_bits(0, 16, None, None) == E

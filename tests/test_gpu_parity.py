@@ -261,10 +261,15 @@ def test_validate_random_bit_exact():
         flip = r.random((B, maxp)) < 2e-4
         exp[flip] ^= 1
         lens = r.integers(-3, maxp * ps + 5, B).astype(np.int32)
+        n_ab = torch.full((1,), 12345, dtype=torch.int32, device="cuda")   # zeroed by the call
+        first = torch.empty(B, dtype=torch.int32, device="cuda")
         got = kvq.validate(torch.from_numpy(tags.view(np.int32)).cuda(), torch.from_numpy(bt).cuda(),
-                           torch.from_numpy(exp.view(np.int32)).cuda(), torch.from_numpy(lens).cuda(), ps)
-        ref = oracle.validate(tags, bt, exp, lens, ps)
+                           torch.from_numpy(exp.view(np.int32)).cuda(), torch.from_numpy(lens).cuda(), ps,
+                           n_aborted=n_ab, first_bad=first)
+        ref, ref_first = oracle.validate(tags, bt, exp, lens, ps, first_bad=True)
         assert np.array_equal(got.cpu().numpy(), ref), trial
+        assert np.array_equal(first.cpu().numpy(), ref_first), trial
+        assert int(n_ab.item()) == int(ref.sum()), trial
 
 
 def test_tag_bump_matches_oracle():
@@ -308,6 +313,24 @@ def test_e4m3_encode_all_2_32_patterns():
         start = i * chunk
         kvq.e4m3_encode_bits(start, chunk, dev)
         ref = oracle.e4m3_encode_bits_range(start, chunk)
+        got = dev.cpu().numpy()
+        if not np.array_equal(got, ref):
+            bad = np.nonzero(got != ref)[0][:5]
+            raise AssertionError([(hex(start + int(j)), hex(got[j]), hex(ref[j])) for j in bad])
+
+
+@pytest.mark.parametrize("scale", [3.7 / 448, 0.0123])
+def test_e4m3_quantize_division_all_2_32_patterns(scale):
+    """The append's quantize step (device division and conversion) against the
+    oracle's IEEE quotient and integer-arithmetic encoder, every float bit
+    pattern, at two scales."""
+    scale = float(np.float32(scale))
+    chunk = 1 << 28
+    dev = torch.empty(chunk, dtype=torch.uint8, device="cuda")
+    for i in range((1 << 32) // chunk):
+        start = i * chunk
+        kvq.e4m3_quantize_bits(start, chunk, scale, dev)
+        ref = oracle.e4m3_quantize_bits_range(start, chunk, scale)
         got = dev.cpu().numpy()
         if not np.array_equal(got, ref):
             bad = np.nonzero(got != ref)[0][:5]

@@ -53,6 +53,28 @@ def test_validate_matches_brute_force_random():
         assert np.array_equal(got, brute_validate(tags, bt, exp, lens, ps))
 
 
+def test_first_bad_index_matches_brute_force():
+    """Telemetry: the first failing block-table index of each request (-1 if none),
+    against a direct scan in Python."""
+    r = np.random.default_rng(7)
+    for trial in range(50):
+        P, B, maxp, ps = int(r.integers(1, 40)), int(r.integers(1, 9)), int(r.integers(1, 9)), int(r.integers(1, 5))
+        tags = r.integers(0, 3, P).astype(np.uint32)
+        bt = r.integers(-1, P + 1, (B, maxp)).astype(np.int32)
+        exp = r.integers(0, 3, (B, maxp)).astype(np.uint32)
+        lens = r.integers(-3, maxp * ps + 5, B).astype(np.int32)
+        mask, first = oracle.validate(tags, bt, exp, lens, ps, first_bad=True)
+        for b in range(B):
+            n = min(max(int(lens[b]), 0), maxp * ps)
+            want = -1
+            for i in range(-(-n // ps)):
+                p = int(bt[b, i])
+                if not (0 <= p < P) or int(tags[p]) != int(exp[b, i]):
+                    want = i
+                    break
+            assert first[b] == want and mask[b] == (want >= 0), (trial, b)
+
+
 def test_entries_beyond_sequence_are_ignored():
     tags = np.arange(10, dtype=np.uint32)
     bt = np.array([[3, 4, 99]], np.int32)          # third entry is garbage
