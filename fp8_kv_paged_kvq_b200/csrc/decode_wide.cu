@@ -88,7 +88,8 @@ constexpr int kVHalf = kBlk * 128 * 2;                // 64 tokens x 128 dims f1
 constexpr int kVBuf = 2 * kVHalf;                     // one CTA's 256 value dims
 constexpr int kPBuf = kH * kBlk * 2;
 constexpr int kNSc = 4;                               // scale ring entries
-constexpr int kNP = 3;                                // P buffers
+constexpr int kNP = 2;                                // P buffers (freed with V: kPvDone)
+constexpr int kNS = 3;                                // S buffers per MMA stream
 
 constexpr int kOffQ = 0;
 constexpr int kOffK = 74752;                          // kQImage rounded up to 1 KB
@@ -102,11 +103,11 @@ constexpr int kOffFlag = kOffXl + 256 * 4;            // per key stage: page in 
 constexpr int kOffBars = kOffFlag + 16;
 enum {
   // completed in the leader CTA
-  kKFull = 0, kSFree = 3, kQReady = 5, kPReady = 6, kVReady = 8, kOFree = 10,
+  kKFull = 0, kSFree = 3, kQReady = 6, kPReady = 7, kVReady = 9, kOFree = 11,
   // arrive in both CTAs (multicast commits)
-  kSFull = 11, kKFree = 13, kPvDone = 16, kPFree = 18,
+  kSFull = 12, kKFree = 15, kPvDone = 18,
   // local
-  kKPeerFull = 21, kScL = 24, kScR = 27, kQFull = 31, kDrain = 32, kNumBars = 36
+  kKPeerFull = 20, kScL = 23, kScR = 26, kQFull = 30, kDrain = 31, kNumBars = 35
 };
 constexpr int kOffTmem = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = 1024 + kOffTmem + 16;
@@ -114,8 +115,8 @@ static_assert(kQImage <= kOffK, "query image overlaps the key stages");
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 // TMEM columns: O at [0, 256) (value-dim half h of the pair at 128*h), the
-// S accumulator of MMA stream k, buffer s, at 256 + 64*k + 32*s.
-static_assert(256 + 64 * kNumMma <= 512, "tensor memory");
+// S accumulator of MMA stream k, buffer s, at 256 + 32*(kNS*k + s).
+static_assert(256 + 32 * kNS * kNumMma <= 512, "tensor memory");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256;
 
@@ -342,14 +343,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[kKPeerFull + s], 1);
       mbar_init(&bars[kScL + s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kNS; ++s) {
       mbar_init(&bars[kSFree + s], 16);       // per softmax warp, both CTAs
+      mbar_init(&bars[kSFull + s], kNumMma);  // one commit per MMA stream
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[kPReady + s], 16);
       mbar_init(&bars[kVReady + s], 8);
-      mbar_init(&bars[kSFull + s], kNumMma);  // one commit per MMA stream
       mbar_init(&bars[kPvDone + s], kNumMma);
     }
-    for (int s = 0; s < kNP; ++s) mbar_init(&bars[kPFree + s], kNumMma);
     for (int s = 0; s < kNSc; ++s) mbar_init(&bars[kScR + s], 1);
     mbar_init(&bars[kQReady], 2);
     mbar_init(&bars[kOFree], 16);
@@ -450,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int k = warp - kWarpMma;
       const uint32_t sq = smem_u32(smem + kOffQ), sk = smem_u32(smem + kOffK);
       const uint32_t sv = smem_u32(smem + kOffV), sp = smem_u32(smem + kOffP);
-      const uint32_t dcol = tbase + kColS + 64 * k;
+      const uint32_t dcol = tbase + kColS + 32 * kNS * k;
       int32_t j = 0, item = 0;
       bool ok = true;
       // PV of block jj, value-dim half h = k (dims 256h + [0, 256) across
@@ -470,25 +472,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_pair_f16(tbase + 128 * k, pa + ((ks * 32) >> 4), va + ((ks * 4096) >> 4),
                           kIdescPV, (first && ks == 0) ? 0u : 1u);
         }
-        umma_commit_pair(&bars[kPvDone + x]);
-        umma_commit_pair(&bars[kPFree + jj % kNP]);
+        umma_commit_pair(&bars[kPvDone + x]);   // frees V buffer x and P buffer jj % 2
       };
+      // Within a piece QK^T runs two blocks ahead of PV (three S buffers):
+      // QK(j), then PV(j-2); the piece's last two PVs are issued before the
+      // next piece's QK^T, which waits for its query image, loaded only
+      // once the softmax has finished this piece.
       for_pieces(p, u0, u1, [&](int, int32_t, int32_t nt) {
         ok = ok && wait_bar(&bars[kQReady], item & 1);
         for (int32_t i = 0; i < nt && ok; ++i, ++j) {
-          const int s = j % kNK, s2 = j & 1;
+          const int s = j % kNK, s3 = j % kNS;
           ok = wait_bar(&bars[kKFull + s], static_cast<uint32_t>(j / kNK) & 1u);
-          if (ok && k == 0)        // the other CTA's V conversion learns that both stages landed
-            mbar_arrive_remote(mapa_shared(smem_u32(&bars[kKPeerFull + s]), 1));
-          if (ok && j >= 2) ok = wait_bar(&bars[kSFree + s2], ((j >> 1) & 1) ^ 1);
+          if (ok && j >= kNS)
+            ok = wait_bar(&bars[kSFree + s3], static_cast<uint32_t>((j / kNS) & 1) ^ 1u);
           if (!ok) break;
           tc_fence_after();
-          issue_qk(dcol + 32 * s2, sq, sk + s * kStage, k);
-          umma_commit_pair(&bars[kSFull + s2]);
+          issue_qk(dcol + 32 * s3, sq, sk + s * kStage, k);
+          umma_commit_pair(&bars[kSFull + s3]);
           umma_commit_pair(&bars[kKFree + s]);
-          if (i > 0) pv(j - 1, i == 1);
+          if (i >= 2) pv(j - 2, i == 2);
         }
-        if (ok && nt > 0) pv(j - 1, nt == 1);
+        if (ok)
+          for (int32_t r = nt >= 2 ? nt - 2 : 0; r < nt; ++r) pv(j - nt + r, r == 0);
         ++item;
       });
       // every MMA issued has finished before either CTA leaves
@@ -515,8 +520,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = j % kNK, x = j & 1;
         const uint32_t n = static_cast<uint32_t>(j / kNK);
         // both CTAs' stages have landed: the leader's barrier counts both
-        // loads, and the leader's QK-hi issuer forwards its completion
+        // loads, and the leader's first V thread forwards its completion (off
+        // the MMA streams, which a remote arrive would hold up)
         ok = ok && wait_bar(&bars[rank == 0 ? kKFull + s : kKPeerFull + s], n & 1u);
+        if (rank == 0 && vt == 0 && ok)
+          mbar_arrive_remote(mapa_shared(smem_u32(&bars[kKPeerFull + s]), 1));
         ok = ok && wait_bar(&bars[kScL + s], n & 1u);
         const int32_t nvalid = min(kBlk, ntok - (t0 + i) * kBlk);
         if (vt < 32) {
@@ -625,10 +633,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       float m_ref = kNegInf, l_part = 0.0f;
       for (int32_t i = 0; i < nt; ++i, ++j) {
-        const int s2 = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
+        const int s2 = j & 1, s3 = j % kNS;
         const int32_t nvalid = min(kBlk, ntok - (t0 + i) * kBlk);
-        ok = ok && wait_bar(&bars[kSFull + s2], ph);
+        ok = ok && wait_bar(&bars[kSFull + s3], static_cast<uint32_t>(j / kNS) & 1u);
         ok = ok && wait_bar(&bars[kScR + (j & (kNSc - 1))], (j >> 2) & 1);
         ok = __all_sync(0xffffffffu, ok);                   // tcgen05.ld is warp-collective
         tc_fence_after();
@@ -640,8 +647,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k2 = 0; k2 < kNumMma; k2 += 2) {
             uint32_t r0[16], r1[16];
-            tmem_ld16(tl + kColS + 64 * k2 + 32 * s2 + 16 * ch, r0);
-            tmem_ld16(tl + kColS + 64 * (k2 + 1) + 32 * s2 + 16 * ch, r1);
+            tmem_ld16(tl + kColS + 32 * (kNS * k2 + s3) + 16 * ch, r0);
+            tmem_ld16(tl + kColS + 32 * (kNS * (k2 + 1) + s3) + 16 * ch, r1);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 16; ++c) sacc[c] += __uint_as_float(r0[c]) + __uint_as_float(r1[c]);
@@ -682,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* xmj = xm + s2 * 256;
         xmj[part * 64 + hl] = bm;
         named_bar(group_bar, 128);                        // this warp's S loads are done too
-        if (lane == 0 && ok) arrive_leader(&bars[kSFree + s2], rank);
+        if (lane == 0 && ok) arrive_leader(&bars[kSFree + s3], rank);
 #pragma unroll
         for (int o = 1; o < 4; ++o) bm = fmaxf(bm, xmj[((part + o) & 3) * 64 + hl]);
         // Move the reference max when a score exceeds it by 2^8.  The vote keeps
@@ -721,8 +728,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[c >> 1] = pack_f16x2(p0 * sc[c], p1 * sc[c + 1]);
         }
         const int pb = j % kNP;
-        if (j >= kNP)                                     // P buffer free: PV(j - kNP) done
-          ok = ok && wait_bar(&bars[kPFree + pb], static_cast<uint32_t>((j / kNP) & 1) ^ 1u);
+        if (j >= kNP)                                     // P buffer free: PV(j - 2) done
+          ok = ok && wait_bar(&bars[kPvDone + pb], static_cast<uint32_t>((j >> 1) & 1) ^ 1u);
         if (ok) {
 #pragma unroll
           for (int k = 0; k < 2; ++k)
