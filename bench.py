@@ -661,10 +661,14 @@ def run_bulk_append(spec, dev, stream, tokens=65536, iters=20):
     pages = -(-tokens // ps)
     g = torch.Generator(device=dev).manual_seed(11)
     cache = kvq.PagedCache(kvq.FP8_E4M3, kvq.SCALE_HEAD, pages, ps, H, Dk, Dv, device=dev)
-    cache.k_scale.fill_(1.0 / 64)
-    cache.v_scale.fill_(1.0 / 64)
     k = torch.randn(tokens, H, Dk, device=dev, generator=g).to(torch.bfloat16)
     v = torch.randn(tokens, H, Dv, device=dev, generator=g).to(torch.bfloat16)
+    # per-head scales from the data (amax / 448), as at the hand-over; not
+    # powers of two, so every value takes the checked product quotient
+    kvq.scale_from_amax(kvq.amax(k, True), out=cache.k_scale)
+    kvq.scale_from_amax(kvq.amax(v, True), out=cache.v_scale)
+    pow2 = bool(((cache.k_scale.view(torch.int32) & 0x7FFFFF) == 0).any() or
+                ((cache.v_scale.view(torch.int32) & 0x7FFFFF) == 0).any())
     perm = torch.randperm(pages, device=dev, generator=g).to(torch.int32)
     t = torch.arange(tokens, device=dev, dtype=torch.int32)
     slots = (perm[t // ps] * ps + t % ps).contiguous()
@@ -678,7 +682,8 @@ def run_bulk_append(spec, dev, stream, tokens=65536, iters=20):
     del gr
     return {"tokens": tokens, "ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
             "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm, "peak_kind": kind,
-            "bytes": nbytes, "note": "bf16 K/V read + e4m3 codes written + slot mapping"}
+            "bytes": nbytes, "note": "bf16 K/V read + e4m3 codes written + slot mapping",
+            "scales": "per head, amax / 448 of the data" + (" (some powers of two)" if pow2 else "")}
 
 
 def run_sweep(args):

@@ -65,16 +65,74 @@ __global__ void scale_from_amax_kernel(const float* __restrict__ amax, float* __
 // and then the V row (for head dims 128 that is one group per lane), so a
 // half-warp writes 128 contiguous code bytes with 8-byte stores.
 // ---------------------------------------------------------------------------
-// Eight bf16 values to eight E4M3 codes of v / s (IEEE binary32 division,
-// then rounding to nearest even with saturation in the conversion).
-__device__ __forceinline__ uint2 quantize8(const uint4 a, float s) {
+// The quotient v / s that the E4M3 encode rounds, without a hardware
+// division per value.  r = RN(1/s) is worked out once per scale, and for
+// |s| in [2^-40, 2^40] q = RN(v r) stands in for RN(v / s):
+//  * s a power of two: r = 1/s exactly, so q = RN(v / s).
+//  * otherwise v r = (v / s)(1 + e) with |e| <= 2^-24, so q and RN(v / s)
+//    are at most three units in the last place apart.  The encode rounds at
+//    values of at most five significant bits (midpoints of E4M3 neighbours
+//    and of its subnormal steps), whose low 19 mantissa bits are zero; where
+//    none is within four units of q (the low 19 bits of q, plus 4, exceed 8
+//    modulo 2^19) both encode alike.  Infinities and NaNs encode alike on
+//    both sides (saturated, or the NaN code).
+// The rare value near such a boundary, and any scale out of the range, takes
+// the IEEE division instead.
+struct QuantScale {
+  float s, r;
+  int kind;          // 0: divide; 1: product, exact; 2: product where the window check passes
+};
+
+__device__ __forceinline__ QuantScale quant_scale(float s) {
+  const float as = fabsf(s);
+  const bool in = as >= 0x1p-40f && as <= 0x1p40f;               // NaN: out
+  const bool pow2 = (__float_as_uint(s) & 0x7FFFFFu) == 0u;
+  return QuantScale{s, __frcp_rn(s), in ? (pow2 ? 1 : 2) : 0};
+}
+
+// Eight bf16 values times r, to eight E4M3 codes; with kWindow, win takes the
+// minimum over the values of ((bits(q) + 4) mod 2^19).
+template <bool kWindow>
+__device__ __forceinline__ uint2 quantize8_mul(const uint4 a, float r, uint32_t& win) {
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+  uint32_t pairs[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float lo = bf16lo_to_f32(w[k]) * r, hi = bf16hi_to_f32(w[k]) * r;
+    if (kWindow)
+      win = min(win, min((__float_as_uint(lo) + 4u) & 0x7FFFFu, (__float_as_uint(hi) + 4u) & 0x7FFFFu));
+    pairs[k] = f32x2_to_e4m3x2(lo, hi);                         // lo code | hi code << 8
+  }
+  return make_uint2(pairs[0] | (pairs[1] << 16), pairs[2] | (pairs[3] << 16));
+}
+
+// The same codes through the IEEE division (a call of its own, so it costs
+// nothing where it is skipped).
+__device__ __noinline__ uint2 quantize8_div(const uint4 a, float s) {
   const uint32_t w[4] = {a.x, a.y, a.z, a.w};
   uint32_t pairs[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k)
     pairs[k] = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[k]), s),
-                               __fdiv_rn(bf16hi_to_f32(w[k]), s));   // lo code | hi code << 8
+                               __fdiv_rn(bf16hi_to_f32(w[k]), s));
   return make_uint2(pairs[0] | (pairs[1] << 16), pairs[2] | (pairs[3] << 16));
+}
+
+// Eight bf16 values to eight E4M3 codes of v / s: E(RN(v / s)), rounding to
+// nearest even with saturation in the conversion.
+__device__ __forceinline__ uint2 quantize8(const uint4 a, const QuantScale& d) {
+  uint32_t win = 0xFFFFFFFFu;
+  if (d.kind == 1) return quantize8_mul<false>(a, d.r, win);
+  const uint2 c = quantize8_mul<true>(a, d.r, win);
+  return d.kind == 2 && win > 8u ? c : quantize8_div(a, d.s);
+}
+
+// One float value, the same way (the exhaustive check of the quotient).
+__device__ __forceinline__ uint32_t quantize1(float v, const QuantScale& d) {
+  float q = v * d.r;
+  const bool near = ((__float_as_uint(q) + 4u) & 0x7FFFFu) <= 8u;
+  if (d.kind == 0 || (d.kind == 2 && near)) q = __fdiv_rn(v, d.s);
+  return f32x2_to_e4m3x2(q, 0.0f) & 0xFFu;
 }
 
 __device__ __forceinline__ float amax8(const uint4 a) {
@@ -87,7 +145,7 @@ __device__ __forceinline__ float amax8(const uint4 a) {
 }
 
 constexpr int kAppendWarps = 8;
-constexpr int kRowsPerWarp = 4;      // (token, head) rows per warp in the batched case
+constexpr int kRowsPerWarp = 8;      // (token, head) rows per warp in the batched case
 
 struct AppendArgs {
   CacheView c;
@@ -104,46 +162,69 @@ struct AppendArgs {
 // The common case: K and V rows of at most 32 eight-value groups together
 // (head dims up to 128) with a per-tensor or per-head scale.  A warp takes
 // kRowsPerWarp rows and issues all their loads before converting any, so
-// four 16-byte loads per lane are in flight.  Rows run token-major within a
-// head (row r: head r / T, token r % T), so a warp writes consecutive slots
-// of one head: contiguous bytes when the tokens' slots are consecutive.
+// eight 16-byte loads per lane are in flight.  Warp w takes head w % Hkv of
+// tokens kRowsPerWarp * (w / Hkv) + [0, kRowsPerWarp): it writes consecutive
+// slots of one head (contiguous bytes when the tokens' slots are
+// consecutive), and the warps of a block, consecutive heads of the same
+// tokens, read one contiguous span of the new K and V rows.
 template <bool FP8>
-__device__ __forceinline__ void append_rows_batched(const AppendArgs& a, int64_t row0, int lane) {
+__device__ __forceinline__ void append_rows_batched(const AppendArgs& a, int32_t w, int lane) {
   const CacheView& c = a.c;
-  const int64_t rows = static_cast<int64_t>(a.T) * c.Hkv;
+  const int32_t h = w % c.Hkv;
+  const int32_t tb = (w / c.Hkv) * kRowsPerWarp;
   const int32_t nk = c.Dk / 8, nv = c.Dv / 8;
   const bool isk = lane < nk, active = lane < nk + nv;
   const int32_t e = 8 * (isk ? lane : lane - nk);
   uint4 x[kRowsPerWarp];
-  int64_t prow[kRowsPerWarp];
-  int32_t hh[kRowsPerWarp];
 #pragma unroll
   for (int i = 0; i < kRowsPerWarp; ++i) {
-    const int64_t r = row0 + i;
-    prow[i] = -1;
-    hh[i] = 0;
     x[i] = make_uint4(0, 0, 0, 0);
-    if (r < rows) {
-      const int32_t h = static_cast<int32_t>(r / a.T), t = static_cast<int32_t>(r % a.T);
-      const int64_t slot = a.slot_mapping[t];
-      hh[i] = h;
-      if (slot >= 0 && slot < static_cast<int64_t>(c.P) * c.ps)
-        prow[i] = ((slot / c.ps) * c.Hkv + h) * c.ps + slot % c.ps;
-      if (active)
-        x[i] = __ldg(reinterpret_cast<const uint4*>(
-            (isk ? a.k_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dk
-                 : a.v_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dv) + e));
+    if (tb + i < a.T && active) {
+      const int64_t t = tb + i;
+      x[i] = __ldg(reinterpret_cast<const uint4*>(
+          (isk ? a.k_new + (t * c.Hkv + h) * c.Dk : a.v_new + (t * c.Hkv + h) * c.Dv) + e));
+    }
+  }
+  // Lane i works out token tb + i's cache row (-1: none) in 32-bit
+  // arithmetic; the warp reads it by shuffle.
+  int64_t my_row = -1;
+  if (lane < kRowsPerWarp && tb + lane < a.T) {
+    const int32_t slot = __ldg(a.slot_mapping + tb + lane);
+    if (slot >= 0 && static_cast<int64_t>(slot) < static_cast<int64_t>(c.P) * c.ps) {
+      const uint32_t pg = static_cast<uint32_t>(slot) / static_cast<uint32_t>(c.ps);
+      const uint32_t o = static_cast<uint32_t>(slot) - pg * static_cast<uint32_t>(c.ps);
+      my_row = (static_cast<int64_t>(pg) * c.Hkv + h) * c.ps + o;
+    }
+  }
+  int64_t prow[kRowsPerWarp];
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp; ++i) prow[i] = __shfl_sync(0xffffffffu, my_row, i);
+  uint2 code[FP8 ? kRowsPerWarp : 1];
+  if (FP8) {
+    // all rows' codes by the product; a lane with a value near a rounding
+    // boundary (rare) divides them all
+    QuantScale qs{1.0f, 1.0f, 1};
+    if (active) qs = quant_scale((isk ? c.k_scale : c.v_scale)[c.scale_mode == 0 ? 0 : h]);
+    uint32_t win = 0xFFFFFFFFu;
+    if (qs.kind == 1) {
+#pragma unroll
+      for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_mul<false>(x[i], qs.r, win);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_mul<true>(x[i], qs.r, win);
+      if (qs.kind == 0 || win <= 8u) {
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_div(x[i], qs.s);
+      }
     }
   }
 #pragma unroll
   for (int i = 0; i < kRowsPerWarp; ++i) {
     if (prow[i] < 0 || !active) continue;
     if (FP8) {
-      const float* sc = isk ? c.k_scale : c.v_scale;
-      const float s = sc[c.scale_mode == 0 ? 0 : hh[i]];
       uint8_t* dst = static_cast<uint8_t*>(isk ? c.k_pages : c.v_pages) +
                      prow[i] * (isk ? c.Dk : c.Dv) + e;
-      *reinterpret_cast<uint2*>(dst) = quantize8(x[i], s);
+      *reinterpret_cast<uint2*>(dst) = code[FP8 ? i : 0];
     } else {
       uint16_t* dst = static_cast<uint16_t*>(isk ? c.k_pages : c.v_pages) +
                       prow[i] * (isk ? c.Dk : c.Dv) + e;
@@ -154,7 +235,7 @@ __device__ __forceinline__ void append_rows_batched(const AppendArgs& a, int64_t
 
 
 
-__global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(kAppendWarps * 32, 4) append_kernel(AppendArgs a) {
   pdl_trigger();            // the tag check may start loading its block-table entries
   const CacheView& c = a.c;
   if (static_cast<int32_t>(blockIdx.x) >= a.token_blocks) {
@@ -166,20 +247,20 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a)
   }
   const int lane = threadIdx.x & 31;
   if (a.batched > 1) {
-    const int64_t row0 =
-        (static_cast<int64_t>(blockIdx.x) * kAppendWarps + (threadIdx.x >> 5)) * kRowsPerWarp;
-    if (c.fp8) append_rows_batched<true>(a, row0, lane);
-    else append_rows_batched<false>(a, row0, lane);
+    const int32_t w = static_cast<int32_t>(blockIdx.x) * kAppendWarps + (threadIdx.x >> 5);
+    if (c.fp8) append_rows_batched<true>(a, w, lane);
+    else append_rows_batched<false>(a, w, lane);
     return;
   }
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kAppendWarps + (threadIdx.x >> 5);
-  if (row >= static_cast<int64_t>(a.T) * c.Hkv) return;
-  const int32_t t = static_cast<int32_t>(row / c.Hkv);
-  const int32_t h = static_cast<int32_t>(row % c.Hkv);
-  const int64_t slot = a.slot_mapping[t];
-  if (slot < 0 || slot >= static_cast<int64_t>(c.P) * c.ps) return;
-  const int64_t p = slot / c.ps, o = slot % c.ps;
-  const int64_t prow = (p * c.Hkv + h) * c.ps + o;   // [P][Hkv][ps] row index
+  const uint32_t row = blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
+  if (static_cast<int64_t>(row) >= static_cast<int64_t>(a.T) * c.Hkv) return;
+  const int32_t t = static_cast<int32_t>(row / static_cast<uint32_t>(c.Hkv));
+  const int32_t h = static_cast<int32_t>(row) - t * c.Hkv;
+  const int32_t slot = a.slot_mapping[t];
+  if (slot < 0 || static_cast<int64_t>(slot) >= static_cast<int64_t>(c.P) * c.ps) return;
+  const uint32_t pg = static_cast<uint32_t>(slot) / static_cast<uint32_t>(c.ps);
+  const uint32_t o = static_cast<uint32_t>(slot) - pg * static_cast<uint32_t>(c.ps);
+  const int64_t prow = (static_cast<int64_t>(pg) * c.Hkv + h) * c.ps + o;   // [P][Hkv][ps] row
   const int32_t nk = c.Dk / 8, nv = c.v_pages == nullptr ? 0 : c.Dv / 8;
   const uint16_t* ksrc = a.k_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dk;
   const uint16_t* vsrc = a.v_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dv;
@@ -222,11 +303,12 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_kernel(AppendArgs a)
   }
   uint8_t* kdst = static_cast<uint8_t*>(c.k_pages) + prow * c.Dk;
   uint8_t* vdst = nv ? static_cast<uint8_t*>(c.v_pages) + prow * c.Dv : nullptr;
+  const QuantScale qk = quant_scale(sk), qv = quant_scale(sv);
   for (int32_t g = lane; g < nk + nv; g += 32) {
     const bool isk = g < nk;
     const int32_t e = 8 * (isk ? g : g - nk);
     const uint4 x = *reinterpret_cast<const uint4*>((isk ? ksrc : vsrc) + e);
-    *reinterpret_cast<uint2*>((isk ? kdst : vdst) + e) = quantize8(x, isk ? sk : sv);
+    *reinterpret_cast<uint2*>((isk ? kdst : vdst) + e) = quantize8(x, isk ? qk : qv);
   }
 }
 
@@ -285,8 +367,10 @@ cudaError_t launch_append(const CacheView& c, const uint16_t* k_new, const uint1
   const bool batched = c.v_pages != nullptr && c.Dk / 8 + c.Dv / 8 <= 32 &&
                        (!c.fp8 || c.scale_mode != 2);
   a.batched = batched ? kRowsPerWarp : 1;
-  const int64_t per_block = static_cast<int64_t>(kAppendWarps) * a.batched;
-  a.token_blocks = static_cast<int32_t>((rows + per_block - 1) / per_block);
+  // batched: one warp per (head, group of kRowsPerWarp tokens); else one per row
+  const int64_t warps =
+      batched ? (static_cast<int64_t>(T) + kRowsPerWarp - 1) / kRowsPerWarp * c.Hkv : rows;
+  a.token_blocks = static_cast<int32_t>((warps + kAppendWarps - 1) / kAppendWarps);
   const int32_t blocks = a.token_blocks + (n_realloc > 0 ? 1 : 0);
   if (blocks == 0) return cudaSuccess;
   append_kernel<<<blocks, kAppendWarps * 32, 0, stream>>>(a);
@@ -299,8 +383,8 @@ __global__ void quantize_bits_kernel(uint32_t start, uint32_t count, float scale
                                      uint8_t* __restrict__ out) {
   const uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= count) return;
-  const float q = __fdiv_rn(__uint_as_float(start + static_cast<uint32_t>(i)), scale);
-  out[i] = static_cast<uint8_t>(f32x2_to_e4m3x2(q, 0.0f) & 0xFFu);
+  out[i] = static_cast<uint8_t>(
+      quantize1(__uint_as_float(start + static_cast<uint32_t>(i)), quant_scale(scale)));
 }
 
 cudaError_t launch_quantize_bits(uint32_t start, uint32_t count, float scale, uint8_t* out,

@@ -100,7 +100,8 @@ constexpr int kOffScR = kOffKSc + kNK * kBlk * 4;     // scale ring read by the 
 constexpr int kOffXm = kOffScR + kNSc * kBlk * 4;
 constexpr int kOffXl = kOffXm + 2 * 256 * 4;         // xm: two blocks' partial maxima
 constexpr int kOffFlag = kOffXl + 256 * 4;            // per key stage: page in range
-constexpr int kOffBars = kOffFlag + 16;
+constexpr int kOffSink = kOffFlag + 16;               // V warps: one word each
+constexpr int kOffBars = kOffSink + 16;
 enum {
   // completed in the leader CTA
   kKFull = 0, kSFree = 3, kQReady = 6, kPReady = 7, kVReady = 9, kOFree = 11,
@@ -555,13 +556,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           e4m3x4_to_f16x2x2_shr8(wv[c].z, f[c][4], f[c][5]);
           e4m3x4_to_f16x2x2_shr8(wv[c].w, f[c][6], f[c][7]);
         }
-        // The conversions above read every loaded register, so once they have
-        // run (the empty asm pins them before the arrivals) this thread's
+        // The OR reads every loaded register and its result is stored, so the
+        // store, and the arrivals issued after it, wait until this thread's
         // loads from both stages have returned; the warp sync covers all lanes.
+        uint32_t dep = 0;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          asm volatile("" ::"r"(f[c][0]), "r"(f[c][1]), "r"(f[c][2]), "r"(f[c][3]), "r"(f[c][4]),
-                       "r"(f[c][5]), "r"(f[c][6]), "r"(f[c][7]));
+        for (int c = 0; c < 8; ++c) dep |= wv[c].x | wv[c].y | wv[c].z | wv[c].w;
+        st_shared_keep(smem_u32(smem + kOffSink) + 4 * (warp - kWarpV), dep);
         __syncwarp();
         if (lane == 0 && ok) {
           mbar_arrive(&bars[kKFree + s]);

@@ -387,6 +387,13 @@ __device__ __forceinline__ void tma_load_4d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// A 32-bit store to this CTA's shared memory that the compiler keeps in
+// program order: storing a value computed from loaded registers makes the
+// thread wait for those loads before anything issued after the store.
+__device__ __forceinline__ void st_shared_keep(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 // 16 bytes from the shared memory of a CTA of the cluster (address from mapa).
 // No memory clobber: volatile asm keeps its order against the barrier waits
 // (also volatile asm), while the compiler may still let several of these

@@ -319,11 +319,12 @@ def test_e4m3_encode_all_2_32_patterns():
             raise AssertionError([(hex(start + int(j)), hex(got[j]), hex(ref[j])) for j in bad])
 
 
-@pytest.mark.parametrize("scale", [3.7 / 448, 0.0123])
+@pytest.mark.parametrize("scale", [3.7 / 448, 0.0123, 2.0 ** -6, 3.0e-11, 7.5e8, 2.0 ** -50])
 def test_e4m3_quantize_division_all_2_32_patterns(scale):
-    """The append's quantize step (device division and conversion) against the
+    """The append's quantize step (device quotient and conversion) against the
     oracle's IEEE quotient and integer-arithmetic encoder, every float bit
-    pattern, at two scales."""
+    pattern: scales with inexact quotients, a power of two (exact ones), the
+    edges of the division-free range and one outside it."""
     scale = float(np.float32(scale))
     chunk = 1 << 28
     dev = torch.empty(chunk, dtype=torch.uint8, device="cuda")
@@ -359,3 +360,45 @@ def test_host_argument_errors():
                                   ctypes.c_void_p(ws.data_ptr()), ws.numel(), 0, None)
         kvq._check("kvq_decode", st)
     assert e.value.status == kvq.KVQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("mode", [kvq.SCALE_TENSOR, kvq.SCALE_HEAD, kvq.SCALE_TOKEN])
+def test_append_every_bf16_pattern(mode):
+    """Every bf16 bit pattern (zeros, subnormals, infinities, NaNs) through
+    kvq_append, with scales inside and outside the range the division-free
+    quotient covers, against the oracle's append: codes and scales bit-exact."""
+    P, ps, H, D = 40, 16, 2, 128
+    T = (1 << 16) // (H * D)                          # 256 tokens: each pattern once in K
+    rng = np.random.default_rng(5)
+    kb = np.arange(1 << 16, dtype=np.uint16).reshape(T, H, D)
+    vb = rng.permutation(np.arange(1 << 16, dtype=np.uint16)).reshape(T, H, D)
+    slots = rng.permutation(P * ps)[:T].astype(np.int32)
+    slots[::37] = -1                                   # some tokens not stored
+    if mode == kvq.SCALE_TENSOR:
+        ks, vs = np.array([0.0123], np.float32), np.array([2.0 ** -50], np.float32)
+    elif mode == kvq.SCALE_HEAD:
+        ks = np.array([3.7 / 448, 1.0e13], np.float32)
+        vs = np.array([2.0 ** -6, 1.0e-40], np.float32)   # the last one subnormal
+    else:
+        ks = vs = None
+    c = kvq.PagedCache(kvq.FP8_E4M3, mode, P, ps, H, D, D)
+    c.k_pages.fill_(0xCD)
+    c.v_pages.fill_(0xCD)
+    if ks is not None:
+        c.k_scale.copy_(torch.from_numpy(ks))
+        c.v_scale.copy_(torch.from_numpy(vs))
+    kt = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16).cuda()
+    vt = torch.from_numpy(vb.view(np.int16)).view(torch.bfloat16).cuda()
+    kvq.append(c, kt, vt, torch.from_numpy(slots).cuda())
+    torch.cuda.synchronize()
+    sshape = (P, H, ps) if mode == kvq.SCALE_TOKEN else ks.shape
+    oc = oracle.Cache(oracle.FP8, mode, P, ps, H, D, D,
+                      np.full((P, H, ps, D), 0xCD, np.uint8), np.full((P, H, ps, D), 0xCD, np.uint8),
+                      np.ones(sshape, np.float32) if ks is None else ks.copy(),
+                      np.ones(sshape, np.float32) if vs is None else vs.copy(),
+                      np.zeros(P, np.uint32))
+    oracle.append(oc, kb, vb, slots)
+    assert np.array_equal(c.k_pages.cpu().numpy(), oc.k_pages)
+    assert np.array_equal(c.v_pages.cpu().numpy(), oc.v_pages)
+    assert np.array_equal(c.k_scale.cpu().numpy().view(np.uint32), oc.k_scale.view(np.uint32))
+    assert np.array_equal(c.v_scale.cpu().numpy().view(np.uint32), oc.v_scale.view(np.uint32))
