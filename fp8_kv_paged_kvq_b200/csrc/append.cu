@@ -65,22 +65,21 @@ __global__ void scale_from_amax_kernel(const float* __restrict__ amax, float* __
 // and then the V row (for head dims 128 that is one group per lane), so a
 // half-warp writes 128 contiguous code bytes with 8-byte stores.
 // ---------------------------------------------------------------------------
-// The quotient v / s that the E4M3 encode rounds, without a hardware
-// division per value.  r = RN(1/s) is worked out once per scale, and for
-// |s| in [2^-40, 2^40] q = RN(v r) stands in for RN(v / s):
-//  * s a power of two: r = 1/s exactly, so q = RN(v / s).
-//  * otherwise v r = (v / s)(1 + e) with |e| <= 2^-24, so q and RN(v / s)
-//    are at most three units in the last place apart.  The encode rounds at
-//    values of at most five significant bits (midpoints of E4M3 neighbours
-//    and of its subnormal steps), whose low 19 mantissa bits are zero; where
-//    none is within four units of q (the low 19 bits of q, plus 4, exceed 8
-//    modulo 2^19) both encode alike.  Infinities and NaNs encode alike on
-//    both sides (saturated, or the NaN code).
-// The rare value near such a boundary, and any scale out of the range, takes
-// the IEEE division instead.
+// The quotient v / s that the E4M3 encode rounds, RN(v / s), without a
+// hardware division per value.  r = RN(1/s) is worked out once per scale.
+//  * s a power of two: r = 1/s exactly and q0 = RN(v r) = RN(v / s).
+//  * otherwise Markstein's correction: q0 = RN(v r), rem = RN(v - q0 s) (one
+//    FMA), q1 = RN(q0 + rem r) (one FMA) equals RN(v / s) for every bf16 v
+//    and every float s whose values and intermediates stay normal; checked
+//    over all 128 bf16 significands x all 2^23 float significands (powers of
+//    two only shift every step).  That holds for |s| in [2^-40, 2^40] and
+//    2^-100 <= |v| < 2^88.  Below 2^-100 the quotient is under 2^-59 and
+//    encodes to a signed zero, whatever its magnitude; the sign is taken
+//    from q0, the sign of v r (zeros included).  From 2^88 up (infinities
+//    and NaNs too) the caller divides.
 struct QuantScale {
   float s, r;
-  int kind;          // 0: divide; 1: product, exact; 2: product where the window check passes
+  int kind;          // 0: divide; 1: product (s a power of two); 2: corrected product
 };
 
 __device__ __forceinline__ QuantScale quant_scale(float s) {
@@ -90,18 +89,28 @@ __device__ __forceinline__ QuantScale quant_scale(float s) {
   return QuantScale{s, __frcp_rn(s), in ? (pow2 ? 1 : 2) : 0};
 }
 
-// Eight bf16 values times r, to eight E4M3 codes; with kWindow, win takes the
-// minimum over the values of ((bits(q) + 4) mod 2^19).
-template <bool kWindow>
-__device__ __forceinline__ uint2 quantize8_mul(const uint4 a, float r, uint32_t& win) {
+template <bool kPow2>
+__device__ __forceinline__ float quant_quotient(float v, float s, float r) {
+  const float q0 = v * r;
+  if (kPow2) return q0;
+  const float rem = fmaf(-q0, s, v);
+  const float q1 = fmaf(rem, r, q0);
+  return __uint_as_float((__float_as_uint(q1) & 0x7FFFFFFFu) | (__float_as_uint(q0) & 0x80000000u));
+}
+
+// Eight bf16 values to eight E4M3 codes by the quotient above.  Without
+// kPow2, big collects the bf16 exponent fields plus 41: bit 15 or 31 set
+// means a value of magnitude 2^88 or more (infinities, NaNs), which the
+// caller sends to the division.
+template <bool kPow2>
+__device__ __forceinline__ uint2 quantize8_mul(const uint4 a, float s, float r, uint32_t& big) {
   const uint32_t w[4] = {a.x, a.y, a.z, a.w};
   uint32_t pairs[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const float lo = bf16lo_to_f32(w[k]) * r, hi = bf16hi_to_f32(w[k]) * r;
-    if (kWindow)
-      win = min(win, min((__float_as_uint(lo) + 4u) & 0x7FFFFu, (__float_as_uint(hi) + 4u) & 0x7FFFFu));
-    pairs[k] = f32x2_to_e4m3x2(lo, hi);                         // lo code | hi code << 8
+    if (!kPow2) big |= (w[k] & 0x7F807F80u) + 0x14801480u;
+    pairs[k] = f32x2_to_e4m3x2(quant_quotient<kPow2>(bf16lo_to_f32(w[k]), s, r),
+                               quant_quotient<kPow2>(bf16hi_to_f32(w[k]), s, r));   // lo | hi << 8
   }
   return make_uint2(pairs[0] | (pairs[1] << 16), pairs[2] | (pairs[3] << 16));
 }
@@ -121,17 +130,20 @@ __device__ __noinline__ uint2 quantize8_div(const uint4 a, float s) {
 // Eight bf16 values to eight E4M3 codes of v / s: E(RN(v / s)), rounding to
 // nearest even with saturation in the conversion.
 __device__ __forceinline__ uint2 quantize8(const uint4 a, const QuantScale& d) {
-  uint32_t win = 0xFFFFFFFFu;
-  if (d.kind == 1) return quantize8_mul<false>(a, d.r, win);
-  const uint2 c = quantize8_mul<true>(a, d.r, win);
-  return d.kind == 2 && win > 8u ? c : quantize8_div(a, d.s);
+  uint32_t big = 0u;
+  if (d.kind == 1) return quantize8_mul<true>(a, d.s, d.r, big);
+  const uint2 c = quantize8_mul<false>(a, d.s, d.r, big);
+  return d.kind == 2 && (big & 0x80008000u) == 0u ? c : quantize8_div(a, d.s);
 }
 
-// One float value, the same way (the exhaustive check of the quotient).
+// One float value, the same way (the exhaustive check of the quotient):
+// the corrected product where its argument holds, else the division.
 __device__ __forceinline__ uint32_t quantize1(float v, const QuantScale& d) {
-  float q = v * d.r;
-  const bool near = ((__float_as_uint(q) + 4u) & 0x7FFFFu) <= 8u;
-  if (d.kind == 0 || (d.kind == 2 && near)) q = __fdiv_rn(v, d.s);
+  const uint32_t ev = (__float_as_uint(v) >> 23) & 0xFFu;
+  float q;
+  if (d.kind == 1) q = quant_quotient<true>(v, d.s, d.r);
+  else if (d.kind == 2 && ev < 215u) q = quant_quotient<false>(v, d.s, d.r);
+  else q = __fdiv_rn(v, d.s);
   return f32x2_to_e4m3x2(q, 0.0f) & 0xFFu;
 }
 
@@ -201,18 +213,18 @@ __device__ __forceinline__ void append_rows_batched(const AppendArgs& a, int32_t
   for (int i = 0; i < kRowsPerWarp; ++i) prow[i] = __shfl_sync(0xffffffffu, my_row, i);
   uint2 code[FP8 ? kRowsPerWarp : 1];
   if (FP8) {
-    // all rows' codes by the product; a lane with a value near a rounding
-    // boundary (rare) divides them all
+    // all rows' codes by the product; a lane holding a value of 2^88 or
+    // more, an infinity or a NaN divides them all
     QuantScale qs{1.0f, 1.0f, 1};
     if (active) qs = quant_scale((isk ? c.k_scale : c.v_scale)[c.scale_mode == 0 ? 0 : h]);
-    uint32_t win = 0xFFFFFFFFu;
+    uint32_t big = 0u;
     if (qs.kind == 1) {
 #pragma unroll
-      for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_mul<false>(x[i], qs.r, win);
+      for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_mul<true>(x[i], qs.s, qs.r, big);
     } else {
 #pragma unroll
-      for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_mul<true>(x[i], qs.r, win);
-      if (qs.kind == 0 || win <= 8u) {
+      for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_mul<false>(x[i], qs.s, qs.r, big);
+      if (qs.kind == 0 || (big & 0x80008000u) != 0u) {
 #pragma unroll
         for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_div(x[i], qs.s);
       }
