@@ -33,10 +33,13 @@ __global__ void __launch_bounds__(kValThreads)
                     int32_t ps, int32_t max_pages, uint8_t* __restrict__ abort_mask,
                     int32_t* __restrict__ n_aborted, int32_t* __restrict__ first_bad) {
   // Launched as a programmatic dependent of the previous kernel (kvq_append
-  // in a decode step): the launch overlaps that kernel, and every global
-  // read here comes after it has finished.
+  // in a decode step), whose launch it overlaps.  The sequence lengths, the
+  // block table and the expected tags are read before the wait: a kernel
+  // that lets this one start early (kvq_append, which triggers at its start)
+  // never writes them, and whatever wrote them earlier in the stream finished
+  // before that kernel began.  The live tags, which kvq_append bumps, are
+  // read only after the wait.
   pdl_trigger();
-  pdl_wait();
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
@@ -50,10 +53,9 @@ __global__ void __launch_bounds__(kValThreads)
   const int32_t npages = static_cast<int32_t>((n + ps - 1) / ps);
   const int32_t* bt = block_table + static_cast<int64_t>(b) * max_pages;
   const uint32_t* ex = expected + static_cast<int64_t>(b) * max_pages;
-  int32_t bad = INT32_MAX;          // smallest failing block-table index seen
-  for (int32_t base = rank * kPerCta; base < npages; base += C * kPerCta) {
-    int32_t page[kPerThread];
-    uint32_t want[kPerThread];
+  int32_t page[kPerThread];
+  uint32_t want[kPerThread];
+  auto load_round = [&](int32_t base) {
 #pragma unroll
     for (int k = 0; k < kPerThread; ++k) {
       const int32_t i = base + k * kValThreads + threadIdx.x;   // coalesced
@@ -64,6 +66,12 @@ __global__ void __launch_bounds__(kValThreads)
         want[k] = ex[i];
       }
     }
+  };
+  load_round(rank * kPerCta);
+  pdl_wait();
+  int32_t bad = INT32_MAX;          // smallest failing block-table index seen
+  for (int32_t base = rank * kPerCta; base < npages; base += C * kPerCta) {
+    if (base != rank * kPerCta) load_round(base);
 #pragma unroll
     for (int k = 0; k < kPerThread; ++k) {
       const int32_t i = base + k * kValThreads + threadIdx.x;

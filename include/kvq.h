@@ -159,8 +159,12 @@ kvq_status kvq_append(const kvq_cache* cache, const void* k_new, const void* v_n
  *   n_aborted   i32 [1]: set to the number of aborted requests (zeroed on
  *               the stream first, so it needs no initialisation);
  *   first_bad   i32 [B]: the smallest failing index i of each request, or -1.
- * Launched as a programmatic dependent of the previous kernel on the stream;
- * it reads nothing before that kernel has finished.
+ * Launched as a programmatic dependent of the previous kernel on the stream.
+ * It reads seq_lens, block_table and expected_tags while that kernel may
+ * still run, and page_tags only after it has finished: the kernel launched
+ * just before on the same stream must not write the first three (kvq_append,
+ * the usual predecessor, never does; copies and earlier kernels are
+ * complete before it starts).
  */
 kvq_status kvq_validate(const uint32_t* page_tags, int32_t num_pages, const int32_t* block_table,
                         const uint32_t* expected_tags, const int32_t* seq_lens,
