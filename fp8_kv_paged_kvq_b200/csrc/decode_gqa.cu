@@ -190,8 +190,11 @@ struct GqaKernel {
   static size_t smem_bytes(int B) { return 1024 + kOffPre + static_cast<size_t>(B + 1) * 4; }
 };
 
+// Registers: two CTAs per SM for one n-tile (128 per thread), and for the FP8
+// kernel 120, so that the tag check launched before it (128 threads of 32
+// registers per SM) fits beside its two CTAs and they start while it runs.
 template <bool FP8, int D, int NT, int NW, int S>
-__global__ void __launch_bounds__(NW * 32, (NT == 1 ? 2 : 1))
+__global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap k_map,
                       const __grid_constant__ CUtensorMap v_map, const GqaParams p) {
   using K = GqaKernel<FP8, D, NT, NW, S>;

@@ -101,15 +101,208 @@ __global__ void __launch_bounds__(kValThreads)
   cluster.sync();   // every CTA's flag stays alive until rank 0 has read it
 }
 
+// ---------------------------------------------------------------------------
+// The same check for batches of up to kFlatMaxB requests, sized so that it
+// shares each SM with the decode kernel that follows it: one CTA of 128
+// threads and at most 32 registers per SM (the decode kernel's two CTAs leave
+// 4,096 registers), so the decode CTAs are resident, past their prologue and
+// waiting while the check runs.  The block-table entries of all requests form
+// one flat index space (request b owns [pre[b], pre[b+1])); CTA g takes the
+// g-th of gridDim.x equal slices, so long and short requests cost alike.
+// Failures go to a per-request word in device memory (the largest
+// INT32_MAX - i over failing entries i, so 0 means none); the last CTA to
+// finish (a ticket that also counts the CTAs that saw a failure) writes every
+// request's mask byte and telemetry and puts the words and the ticket back to
+// 0, reading the words only when some CTA failed.  The words are shared by
+// the library's calls on one device, so these calls must not overlap.
+// ---------------------------------------------------------------------------
+constexpr int kFlatThreads = 128;
+constexpr int kFlatPer = 8;                 // entries per thread and round
+constexpr int kFlatMaxB = 4096;             // prefix of B + 1 ints in shared memory
+
+__device__ int32_t g_val_acc[kFlatMaxB];
+__device__ uint32_t g_val_ticket = 0;       // (CTAs that failed << 16) | CTAs done
+
+__global__ void __maxnreg__(32)
+    validate_flat_kernel(const uint32_t* __restrict__ tags, int32_t P,
+                         const int32_t* __restrict__ block_table,
+                         const uint32_t* __restrict__ expected,
+                         const int32_t* __restrict__ seq_lens, int32_t ps, int32_t B,
+                         int32_t max_pages, uint8_t* __restrict__ abort_mask,
+                         int32_t* __restrict__ n_aborted, int32_t* __restrict__ first_bad) {
+  // The same programmatic-dependent-launch contract as validate_kernel: the
+  // sequence lengths, block table and expected tags are read before the
+  // wait, the live tags after it.
+  pdl_trigger();
+  __shared__ int32_t pre[kFlatMaxB + 1];
+  __shared__ int32_t warp_sum[kFlatThreads / 32];
+  __shared__ uint32_t ticket;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t cap = static_cast<int64_t>(max_pages) * ps;
+  // pages per request, then an exclusive prefix (each thread a run of requests)
+  const int per = (B + kFlatThreads - 1) / kFlatThreads;
+  const int r0 = min(B, tid * per), r1 = min(B, r0 + per);
+  int32_t run = 0;
+  for (int b = r0; b < r1; ++b) {
+    int64_t n = seq_lens[b];
+    n = n < 0 ? 0 : (n > cap ? cap : n);
+    pre[b] = static_cast<int32_t>((n + ps - 1) / ps);
+    run += pre[b];
+  }
+  int32_t incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  int32_t base = incl - run;
+  for (int w = 0; w < warp; ++w) base += warp_sum[w];
+  for (int b = r0; b < r1; ++b) {
+    const int32_t np = pre[b];
+    pre[b] = base;
+    base += np;
+  }
+  if (tid == kFlatThreads - 1) pre[B] = base;
+  __syncthreads();
+  const int64_t E = pre[B];
+  const int32_t f0 = static_cast<int32_t>(E * blockIdx.x / gridDim.x);
+  const int32_t f1 = static_cast<int32_t>(E * (blockIdx.x + 1) / gridDim.x);
+  // entry f -> (request b, index i within its row): the largest b >= from
+  // with pre[b] <= f, by doubling steps from `from` and then halving
+  auto locate = [&](int32_t f, int from, int32_t& b, int32_t& i) {
+    int lo = from, step = 1;
+    while (lo + step < B && pre[lo + step] <= f) {
+      lo += step;
+      step <<= 1;
+    }
+    for (step >>= 1; step > 0; step >>= 1)
+      if (lo + step < B && pre[lo + step] <= f) lo += step;
+    b = lo;
+    i = f - pre[lo];
+  };
+  int32_t page[kFlatPer];
+  uint32_t want[kFlatPer];
+  auto load_round = [&](int32_t r) {
+    int32_t b = 0, i;
+#pragma unroll
+    for (int k = 0; k < kFlatPer; ++k) {
+      const int32_t f = r + k * kFlatThreads + tid;
+      page[k] = 0;
+      want[k] = 0;
+      if (f < f1) {
+        locate(f, b, b, i);                 // entries grow with k: start from the last
+        const int64_t e = static_cast<int64_t>(b) * max_pages + i;
+        page[k] = block_table[e];
+        want[k] = expected[e];
+      }
+    }
+  };
+  load_round(f0);
+  // The live tags may still change (kvq_append bumps reallocated pages), but
+  // their lines can come into L2 now: the loads after the wait then hit L2
+  // instead of making scattered DRAM reads on the step's critical path.
+#pragma unroll
+  for (int k = 0; k < kFlatPer; ++k)
+    if (page[k] >= 0 && page[k] < P) prefetch_l2(tags + page[k]);
+  pdl_wait();
+  int fail = 0;
+  for (int32_t r = f0; r < f1; r += kFlatPer * kFlatThreads) {
+    if (r != f0) load_round(r);
+    // all of the round's tag loads first (no store between them), failures
+    // as bits; the rare failing entry then goes to its request's word
+    uint32_t bits = 0;
+#pragma unroll
+    for (int k = 0; k < kFlatPer; ++k) {
+      const int32_t f = r + k * kFlatThreads + tid;
+      const int32_t p = page[k];
+      const bool in = p >= 0 && p < P;
+      const uint32_t live = in ? tags[in ? p : 0] : 0u;
+      if (f < f1 && (!in || live != want[k])) bits |= 1u << k;
+    }
+    if (bits != 0) {
+#pragma unroll 1
+      for (int k = 0; k < kFlatPer; ++k) {
+        if ((bits >> k) & 1u) {
+          int32_t b, i;
+          locate(r + k * kFlatThreads + tid, 0, b, i);
+          atomicMax(&g_val_acc[b], INT32_MAX - i);
+        }
+      }
+      fail = 1;
+    }
+  }
+  if (fail) __threadfence();                // this thread's failure words before the ticket
+  const int any = __syncthreads_or(fail);
+  if (tid == 0) {
+    ticket = atomicAdd(&g_val_ticket, 1u + (any ? 0x10000u : 0u)) + (any ? 0x10000u : 0u);
+  }
+  __syncthreads();
+  const uint32_t t = ticket;
+  if ((t & 0xFFFFu) != gridDim.x - 1) return;
+  // last CTA: every other CTA's failure words are visible
+  __threadfence();
+  const bool some = (t >> 16) != 0;
+  int32_t cnt = 0;
+  for (int b = tid; b < B; b += kFlatThreads) {
+    const int32_t v = some ? atomicExch(&g_val_acc[b], 0) : 0;
+    abort_mask[b] = v != 0 ? 1 : 0;
+    if (first_bad != nullptr) first_bad[b] = v != 0 ? INT32_MAX - v : -1;
+    cnt += v != 0 ? 1 : 0;
+  }
+  if (n_aborted != nullptr) {
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (lane == 0) warp_sum[warp] = cnt;
+    __syncthreads();
+    if (tid == 0) {
+      int32_t total = 0;
+      for (int w = 0; w < kFlatThreads / 32; ++w) total += warp_sum[w];
+      *n_aborted = total;
+    }
+  }
+  if (tid == 0) g_val_ticket = 0;
+}
+
 cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* block_table,
                             const uint32_t* expected, const int32_t* seq_lens, int32_t ps,
                             int32_t B, int32_t max_pages, uint8_t* abort_mask,
                             int32_t* n_aborted, int32_t* first_bad, cudaStream_t stream) {
+  if (B == 0) {
+    if (n_aborted == nullptr) return cudaSuccess;
+    return cudaMemsetAsync(n_aborted, 0, sizeof(int32_t), stream);
+  }
+  if (B <= kFlatMaxB && static_cast<int64_t>(B) * max_pages <= 0x7fffffff) {
+    static int sms[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (sms[dev] == 0) {
+      e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+      // keep the SM's shared memory at its largest split while this runs,
+      // so the decode CTAs (about 100 KB each) fit beside it
+      e = cudaFuncSetAttribute(validate_flat_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sms[dev]));
+    cfg.blockDim = dim3(kFlatThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, validate_flat_kernel, tags, P, block_table, expected,
+                              seq_lens, ps, B, max_pages, abort_mask, n_aborted, first_bad);
+  }
   if (n_aborted != nullptr) {
     const cudaError_t e = cudaMemsetAsync(n_aborted, 0, sizeof(int32_t), stream);
     if (e != cudaSuccess) return e;
   }
-  if (B == 0) return cudaSuccess;
   int C = (max_pages + kPerCta - 1) / kPerCta;
   C = C < 1 ? 1 : (C > kMaxCluster ? kMaxCluster : C);
   if (static_cast<int64_t>(B) * C > 0x7fffffff) return cudaErrorInvalidValue;

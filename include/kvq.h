@@ -156,8 +156,8 @@ kvq_status kvq_append(const kvq_cache* cache, const void* k_new, const void* v_n
  * Optional telemetry (device pointers, NULL to skip), because the pages name
  * the mismatch rate as the quantity to watch ([remio] "Sicherheit
  * gemeinsamer KV-Caches wird zum Produktionsthema"):
- *   n_aborted   i32 [1]: set to the number of aborted requests (zeroed on
- *               the stream first, so it needs no initialisation);
+ *   n_aborted   i32 [1]: set to the number of aborted requests (needs no
+ *               initialisation);
  *   first_bad   i32 [B]: the smallest failing index i of each request, or -1.
  * Launched as a programmatic dependent of the previous kernel on the stream.
  * It reads seq_lens, block_table and expected_tags while that kernel may
@@ -165,6 +165,14 @@ kvq_status kvq_append(const kvq_cache* cache, const void* k_new, const void* v_n
  * just before on the same stream must not write the first three (kvq_append,
  * the usual predecessor, never does; copies and earlier kernels are
  * complete before it starts).
+ * Batches of up to 4,096 requests (and B * max_pages < 2^31) run as one CTA
+ * of 128 threads per SM over all requests' entries, small enough to share
+ * each SM with the decode launch that follows, whose CTAs then start while
+ * the check runs.  Its CTAs combine failures through a small accumulator in
+ * the library's device memory, which returns to zero at the end of each
+ * call: on one device, such calls must not run at the same time (on
+ * different streams).  Larger batches use one cluster of up to 8 CTAs per
+ * request and have no such restriction.
  */
 kvq_status kvq_validate(const uint32_t* page_tags, int32_t num_pages, const int32_t* block_table,
                         const uint32_t* expected_tags, const int32_t* seq_lens,

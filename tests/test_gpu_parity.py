@@ -272,6 +272,32 @@ def test_validate_random_bit_exact():
         assert int(n_ab.item()) == int(ref.sum()), trial
 
 
+@pytest.mark.parametrize("B", [1, 4095, 4096, 4097, 6000])
+def test_validate_batch_sizes_and_reset(B):
+    """Batches on both sides of the flat / per-request-cluster switch, each
+    checked after a failing call so that state carried between calls would
+    show: failing, then clean, then failing again."""
+    r = np.random.default_rng(B)
+    P, maxp, ps = 5000, 6, 16
+    tags = r.integers(0, 1 << 32, P, dtype=np.uint64).astype(np.uint32)
+    bt = r.integers(0, P, (B, maxp)).astype(np.int32)
+    lens = r.integers(0, maxp * ps + 1, B).astype(np.int32)
+    clean = tags[bt].copy()
+    stale = clean.copy()
+    hit = r.integers(0, B, max(1, B // 50))
+    stale[hit, r.integers(0, maxp, hit.size)] ^= 1
+    dev = lambda a: torch.from_numpy(a).cuda()
+    for exp in (stale, clean, stale):
+        n_ab = torch.full((1,), -7, dtype=torch.int32, device="cuda")
+        first = torch.full((B,), -9, dtype=torch.int32, device="cuda")
+        got = kvq.validate(dev(tags.view(np.int32)), dev(bt), dev(exp.view(np.int32)), dev(lens), ps,
+                           n_aborted=n_ab, first_bad=first)
+        ref, ref_first = oracle.validate(tags, bt, exp, lens, ps, first_bad=True)
+        assert np.array_equal(got.cpu().numpy(), ref)
+        assert np.array_equal(first.cpu().numpy(), ref_first)
+        assert int(n_ab.item()) == int(ref.sum())
+
+
 def test_tag_bump_matches_oracle():
     P = 50
     tags = np.random.default_rng(1).integers(0, 2**32, P, dtype=np.uint64).astype(np.uint32)
