@@ -287,8 +287,13 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
                                cudaSharedmemCarveoutMaxShared);
       if (e != cudaSuccess) return e;
     }
+    // at most one CTA per SM, and no more than B * max_pages entries need:
+    // one round of kFlatPer loads per thread either way up to 148K entries
+    const int64_t per_cta = static_cast<int64_t>(kFlatThreads) * kFlatPer;
+    const int64_t want = (static_cast<int64_t>(B) * max_pages + per_cta - 1) / per_cta;
+    const int grid = static_cast<int>(want < 1 ? 1 : (want < sms[dev] ? want : sms[dev]));
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(sms[dev]));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kFlatThreads);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
