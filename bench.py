@@ -582,45 +582,60 @@ def run_long(args):
 
 
 def run_e2e(db, args, stream, kv_bytes, world):
-    """Same step through the Python API, step inputs copied from pinned host
-    memory and the result read back, every step."""
-    import fp8_kv_paged_kvq_b200 as kvq
+    """Same step through the public API, its inputs copied from pinned host
+    memory and its results (out, lse, abort mask) read back, every step:
+    - value: two CUDA graphs (DecodeBatch.capture_io_pipelined) replayed in
+      turn; each replay runs one step while copying in the next step's inputs
+      and copying out the previous step's results on side streams;
+    - serial: one graph per step holding its copies, append, validate, decode
+      and read-back in order (DecodeBatch.capture_io_step);
+    - eager: the same calls issued one by one from Python each step."""
     K = args.e2e_steps
-    host_in = {name: t.detach().cpu().pin_memory() for name, t in
-               (("q", db.q), ("k_new", db.k_new), ("v_new", db.v_new), ("slots", db.new_slots),
-                ("seq_lens", db.seq_lens), ("block_table", db.block_table),
-                ("expected", db.expected)) if t is not None}
-    dev_in = {"q": db.q, "k_new": db.k_new, "v_new": db.v_new, "slots": db.new_slots,
-              "seq_lens": db.seq_lens, "block_table": db.block_table, "expected": db.expected}
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    out_h = torch.empty(db.out.shape, dtype=db.out.dtype).pin_memory()
-    lse_h = torch.empty(db.lse.shape, dtype=db.lse.dtype).pin_memory()
-    ab_h = torch.empty(db.abort.shape, dtype=db.abort.dtype).pin_memory()
-    d2h = sum(t.numel() * t.element_size() for t in (out_h, lse_h, ab_h))
+    names = [n for n in db.IO_IN if getattr(db, n) is not None]
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype).pin_memory()
+    host_in = [{n: getattr(db, n).detach().cpu().pin_memory() for n in names} for _ in range(2)]
+    host_out = [{n: pin(getattr(db, n)) for n in db.IO_OUT} for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in[0].values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
 
     def one():
-        for name, h in host_in.items():
-            dev_in[name].copy_(h, non_blocking=True)
+        for n, h in host_in[0].items():
+            getattr(db, n).copy_(h, non_blocking=True)
         db.step(check_tags=True, stream=stream)
-        out_h.copy_(db.out, non_blocking=True)
-        lse_h.copy_(db.lse, non_blocking=True)
-        ab_h.copy_(db.abort, non_blocking=True)
+        for n, h in host_out[0].items():
+            h.copy_(getattr(db, n), non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        for _ in range(5):
-            one()
+    def timed(fns):
+        for i in range(6):
+            fns[i % len(fns)]()
         barrier(world)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(K):
-            one()
+        for i in range(K):
+            fns[i % len(fns)]()
         e1.record(stream)
         torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1) / K, world)
-    return {"value": world * kv_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
+        return max_over_ranks(e0.elapsed_time(e1) / K, world)
+
+    with torch.cuda.stream(stream):
+        ms_eager = timed([one])
+        g = db.capture_io_step(host_in[0], host_out[0], stream)
+        ms_serial = timed([g.replay])
+        del g
+        ga, gb = db.capture_io_pipelined(host_in, host_out, stream)
+        ms = timed([ga.replay, gb.replay])
+        del ga, gb
+    gbs = lambda m: world * kv_bytes / (m * 1e-3) / 1e9
+    return {"value": gbs(ms), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "steps": K, "path": "python binding -> C ABI, eager launches"}
+            "steps": K, "path": "python binding -> C ABI; two CUDA graphs in turn, each a step "
+                                "(append, validate, decode) with the next step's host->device "
+                                "copies and the previous step's device->host copies beside it",
+            "serial": {"value": gbs(ms_serial), "ms_per_step": ms_serial,
+                       "path": "one CUDA graph per step: copies in, step, copies out, in order"},
+            "eager": {"value": gbs(ms_eager), "ms_per_step": ms_eager,
+                      "path": "the same calls launched one by one from Python"}}
 
 
 def run_bf16(wl_fp8, args, stream, world, dev):

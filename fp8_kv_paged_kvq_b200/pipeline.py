@@ -89,6 +89,64 @@ class DecodeBatch:
             self.validate(stream)
         return self.decode(use_abort=check_tags, stream=stream)
 
+    def capture_io_step(self, host_in: dict, host_out: dict, stream,
+                        check_tags: bool = True) -> torch.cuda.CUDAGraph:
+        """One step with its host traffic as a CUDA graph.  host_in maps input
+        names (q, k_new, v_new, new_slots, seq_lens, block_table, expected) to
+        pinned host tensors copied in first; host_out maps out, lse and abort to
+        pinned host tensors filled last.  Every replay moves the host buffers'
+        current contents, so a caller refills host_in and replays."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for name, h in host_in.items():
+                getattr(self, name).copy_(h, non_blocking=True)
+            self.step(check_tags, stream=stream)
+            for name, h in host_out.items():
+                h.copy_(getattr(self, name), non_blocking=True)
+        return g
+
+    IO_IN = ("q", "k_new", "v_new", "new_slots", "seq_lens", "block_table", "expected")
+    IO_OUT = ("out", "lse", "abort")
+
+    def capture_io_pipelined(self, host_in: list, host_out: list, stream):
+        """Two CUDA graphs, replayed alternately, that keep a stream of steps
+        and their host traffic overlapped.  host_in / host_out are two dicts
+        each (pinned host tensors keyed by the names in IO_IN / IO_OUT), one per
+        device buffer set.  Graph k runs a step on buffer set k while side
+        streams copy host_in[1-k] into set 1-k (the next step's inputs) and set
+        1-k's results into host_out[1-k] (the previous step's).  Every replay
+        thus moves one step's inputs and one step's results across the link."""
+        sets = [{n: getattr(self, n) for n in self.IO_IN + self.IO_OUT
+                 if getattr(self, n) is not None}]
+        sets.append({n: t.clone() for n, t in sets[0].items()})
+        side_in, side_out = torch.cuda.Stream(self.device), torch.cuda.Stream(self.device)
+        graphs = []
+        for k in (0, 1):
+            o = 1 - k
+            for n, t in sets[k].items():
+                setattr(self, n, t)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fork = torch.cuda.Event()
+                fork.record(stream)
+                side_in.wait_event(fork)
+                side_out.wait_event(fork)
+                with torch.cuda.stream(side_in):
+                    for n, h in host_in[o].items():
+                        sets[o][n].copy_(h, non_blocking=True)
+                with torch.cuda.stream(side_out):
+                    for n, h in host_out[o].items():
+                        h.copy_(sets[o][n], non_blocking=True)
+                self.step(True, stream=stream)
+                for side in (side_in, side_out):
+                    join = torch.cuda.Event()
+                    join.record(side)
+                    stream.wait_event(join)
+            graphs.append(g)
+        for n, t in sets[0].items():
+            setattr(self, n, t)
+        return graphs
+
 
 class DecodeLoop:
     """The long decode loop on the device.  Every step appends one token per
