@@ -150,7 +150,7 @@ kvq_status kvq_append(const kvq_cache* cache, const void* k_new, const void* v_n
  *   block_table[b][i] outside [0, num_pages) or
  *   page_tags[block_table[b][i]] != expected_tags[b][i],
  * else 0.  Entries of block_table / expected_tags beyond ceil(n/ps) are not
- * read.  One thread-block cluster of up to 8 CTAs checks each request.
+ * read.
  *   block_table i32 [B][max_pages]; expected_tags u32 [B][max_pages];
  *   seq_lens i32 [B]; abort_mask u8 [B] (written).
  * Optional telemetry (device pointers, NULL to skip), because the pages name
