@@ -171,30 +171,40 @@ struct AppendArgs {
   int32_t batched;       // rows per warp: kRowsPerWarp (batched case) or 1
 };
 
-// The common case: K and V rows of at most 32 eight-value groups together
-// (head dims up to 128) with a per-tensor or per-head scale.  A warp takes
-// kRowsPerWarp rows and issues all their loads before converting any, so
-// eight 16-byte loads per lane are in flight.  Warp w takes head w % Hkv of
+// The common case: K and V head dims that are multiples of 16, whose
+// 16-value groups per token (gt = Dk/16 + Dv/16) divide the warp into tp =
+// 32 / gt tokens (2 for d 128, 4 for d 64), and a per-tensor or per-head
+// scale.  A warp takes kRowsPerWarp tokens of one KV head in kRowsPerWarp /
+// tp passes; lane l holds group l % gt (the K row's groups, then the V
+// row's) of token l / gt of each pass: two 16-byte loads of bf16, one
+// 16-byte store of 16 codes.  All loads are issued before any conversion
+// (eight 16-byte loads per lane in flight).  Warp w takes head w % Hkv of
 // tokens kRowsPerWarp * (w / Hkv) + [0, kRowsPerWarp): it writes consecutive
 // slots of one head (contiguous bytes when the tokens' slots are
 // consecutive), and the warps of a block, consecutive heads of the same
 // tokens, read one contiguous span of the new K and V rows.
+constexpr int kMaxPass = 4;          // kRowsPerWarp / tp for tp >= 2
+
 template <bool FP8>
 __device__ __forceinline__ void append_rows_batched(const AppendArgs& a, int32_t w, int lane) {
   const CacheView& c = a.c;
   const int32_t h = w % c.Hkv;
   const int32_t tb = (w / c.Hkv) * kRowsPerWarp;
-  const int32_t nk = c.Dk / 8, nv = c.Dv / 8;
-  const bool isk = lane < nk, active = lane < nk + nv;
-  const int32_t e = 8 * (isk ? lane : lane - nk);
-  uint4 x[kRowsPerWarp];
+  const int32_t gk = c.Dk / 16, gt = gk + c.Dv / 16;
+  const int32_t tp = 32 / gt, passes = kRowsPerWarp / tp;
+  const int32_t sub = lane / gt, g = lane - sub * gt;
+  const bool isk = g < gk;
+  const int32_t e = 16 * (isk ? g : g - gk);
+  uint4 x[kMaxPass][2];
 #pragma unroll
-  for (int i = 0; i < kRowsPerWarp; ++i) {
-    x[i] = make_uint4(0, 0, 0, 0);
-    if (tb + i < a.T && active) {
-      const int64_t t = tb + i;
-      x[i] = __ldg(reinterpret_cast<const uint4*>(
-          (isk ? a.k_new + (t * c.Hkv + h) * c.Dk : a.v_new + (t * c.Hkv + h) * c.Dv) + e));
+  for (int p = 0; p < kMaxPass; ++p) {
+    x[p][0] = x[p][1] = make_uint4(0, 0, 0, 0);
+    const int64_t t = tb + p * tp + sub;
+    if (p < passes && t < a.T) {
+      const uint16_t* src =
+          (isk ? a.k_new + (t * c.Hkv + h) * c.Dk : a.v_new + (t * c.Hkv + h) * c.Dv) + e;
+      x[p][0] = __ldg(reinterpret_cast<const uint4*>(src));
+      x[p][1] = __ldg(reinterpret_cast<const uint4*>(src + 8));
     }
   }
   // Lane i works out token tb + i's cache row (-1: none) in 32-bit
@@ -208,44 +218,51 @@ __device__ __forceinline__ void append_rows_batched(const AppendArgs& a, int32_t
       my_row = (static_cast<int64_t>(pg) * c.Hkv + h) * c.ps + o;
     }
   }
-  int64_t prow[kRowsPerWarp];
-#pragma unroll
-  for (int i = 0; i < kRowsPerWarp; ++i) prow[i] = __shfl_sync(0xffffffffu, my_row, i);
-  uint2 code[FP8 ? kRowsPerWarp : 1];
+  // FP8: the product quotient for every value, or the division for all of
+  // this lane's values when one of them is 2^88 or more, an infinity or a
+  // NaN (bf16 exponent field plus 41 carries into bit 15 or 31), or the
+  // scale is out of the product's range
+  QuantScale qs{1.0f, 1.0f, 1};
+  bool slow = false;
   if (FP8) {
-    // all rows' codes by the product; a lane holding a value of 2^88 or
-    // more, an infinity or a NaN divides them all
-    QuantScale qs{1.0f, 1.0f, 1};
-    if (active) qs = quant_scale((isk ? c.k_scale : c.v_scale)[c.scale_mode == 0 ? 0 : h]);
+    qs = quant_scale((isk ? c.k_scale : c.v_scale)[c.scale_mode == 0 ? 0 : h]);
     uint32_t big = 0u;
-    if (qs.kind == 1) {
 #pragma unroll
-      for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_mul<true>(x[i], qs.s, qs.r, big);
-    } else {
+    for (int p = 0; p < kMaxPass; ++p)
 #pragma unroll
-      for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_mul<false>(x[i], qs.s, qs.r, big);
-      if (qs.kind == 0 || (big & 0x80008000u) != 0u) {
-#pragma unroll
-        for (int i = 0; i < kRowsPerWarp; ++i) code[i] = quantize8_div(x[i], qs.s);
-      }
-    }
+      for (int j = 0; j < 2; ++j)
+        big |= ((x[p][j].x & 0x7F807F80u) + 0x14801480u) | ((x[p][j].y & 0x7F807F80u) + 0x14801480u) |
+               ((x[p][j].z & 0x7F807F80u) + 0x14801480u) | ((x[p][j].w & 0x7F807F80u) + 0x14801480u);
+    slow = qs.kind == 0 || (qs.kind == 2 && (big & 0x80008000u) != 0u);
   }
 #pragma unroll
-  for (int i = 0; i < kRowsPerWarp; ++i) {
-    if (prow[i] < 0 || !active) continue;
+  for (int p = 0; p < kMaxPass; ++p) {
+    const int64_t prow = __shfl_sync(0xffffffffu, my_row, (p * tp + sub) & 31);
+    if (p >= passes || prow < 0) continue;
     if (FP8) {
+      uint2 lo, hi;
+      uint32_t unused = 0u;
+      if (slow) {
+        lo = quantize8_div(x[p][0], qs.s);
+        hi = quantize8_div(x[p][1], qs.s);
+      } else if (qs.kind == 1) {
+        lo = quantize8_mul<true>(x[p][0], qs.s, qs.r, unused);
+        hi = quantize8_mul<true>(x[p][1], qs.s, qs.r, unused);
+      } else {
+        lo = quantize8_mul<false>(x[p][0], qs.s, qs.r, unused);
+        hi = quantize8_mul<false>(x[p][1], qs.s, qs.r, unused);
+      }
       uint8_t* dst = static_cast<uint8_t*>(isk ? c.k_pages : c.v_pages) +
-                     prow[i] * (isk ? c.Dk : c.Dv) + e;
-      *reinterpret_cast<uint2*>(dst) = code[FP8 ? i : 0];
+                     prow * (isk ? c.Dk : c.Dv) + e;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(lo.x, lo.y, hi.x, hi.y);
     } else {
       uint16_t* dst = static_cast<uint16_t*>(isk ? c.k_pages : c.v_pages) +
-                      prow[i] * (isk ? c.Dk : c.Dv) + e;
-      *reinterpret_cast<uint4*>(dst) = x[i];
+                      prow * (isk ? c.Dk : c.Dv) + e;
+      reinterpret_cast<uint4*>(dst)[0] = x[p][0];
+      reinterpret_cast<uint4*>(dst)[1] = x[p][1];
     }
   }
 }
-
-
 
 __global__ void __launch_bounds__(kAppendWarps * 32, 4) append_kernel(AppendArgs a) {
   pdl_trigger();            // the tag check may start loading its block-table entries
@@ -273,7 +290,11 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 4) append_kernel(AppendArgs
   const uint32_t pg = static_cast<uint32_t>(slot) / static_cast<uint32_t>(c.ps);
   const uint32_t o = static_cast<uint32_t>(slot) - pg * static_cast<uint32_t>(c.ps);
   const int64_t prow = (static_cast<int64_t>(pg) * c.Hkv + h) * c.ps + o;   // [P][Hkv][ps] row
-  const int32_t nk = c.Dk / 8, nv = c.v_pages == nullptr ? 0 : c.Dv / 8;
+  // 16-value groups (two 16-byte loads, one 16-byte store of codes) when
+  // both head dims allow, else 8-value groups
+  const bool g16 = c.Dk % 16 == 0 && (c.v_pages == nullptr || c.Dv % 16 == 0);
+  const int32_t gw = g16 ? 16 : 8;
+  const int32_t nk = c.Dk / gw, nv = c.v_pages == nullptr ? 0 : c.Dv / gw;
   const uint16_t* ksrc = a.k_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dk;
   const uint16_t* vsrc = a.v_new + (static_cast<int64_t>(t) * c.Hkv + h) * c.Dv;
   if (!c.fp8) {
@@ -281,9 +302,11 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 4) append_kernel(AppendArgs
     uint16_t* vdst = static_cast<uint16_t*>(c.v_pages) + prow * c.Dv;
     for (int32_t g = lane; g < nk + nv; g += 32) {
       const bool isk = g < nk;
-      const int32_t e = 8 * (isk ? g : g - nk);
-      *reinterpret_cast<uint4*>((isk ? kdst : vdst) + e) =
-          *reinterpret_cast<const uint4*>((isk ? ksrc : vsrc) + e);
+      const int32_t e = gw * (isk ? g : g - nk);
+      const uint4* src = reinterpret_cast<const uint4*>((isk ? ksrc : vsrc) + e);
+      uint4* dst = reinterpret_cast<uint4*>((isk ? kdst : vdst) + e);
+      dst[0] = src[0];
+      if (g16) dst[1] = src[1];
     }
     return;
   }
@@ -298,8 +321,12 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 4) append_kernel(AppendArgs
     // per-token scale: amax over each row, reduced across the warp
     float ak = 0.0f, av = 0.0f;
     for (int32_t g = lane; g < nk + nv; g += 32) {
-      if (g < nk) ak = fmaxf(ak, amax8(*reinterpret_cast<const uint4*>(ksrc + 8 * g)));
-      else av = fmaxf(av, amax8(*reinterpret_cast<const uint4*>(vsrc + 8 * (g - nk))));
+      const bool isk = g < nk;
+      const uint4* src = reinterpret_cast<const uint4*>((isk ? ksrc : vsrc) + gw * (isk ? g : g - nk));
+      float m = amax8(src[0]);
+      if (g16) m = fmaxf(m, amax8(src[1]));
+      if (isk) ak = fmaxf(ak, m);
+      else av = fmaxf(av, m);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -318,9 +345,16 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 4) append_kernel(AppendArgs
   const QuantScale qk = quant_scale(sk), qv = quant_scale(sv);
   for (int32_t g = lane; g < nk + nv; g += 32) {
     const bool isk = g < nk;
-    const int32_t e = 8 * (isk ? g : g - nk);
-    const uint4 x = *reinterpret_cast<const uint4*>((isk ? ksrc : vsrc) + e);
-    *reinterpret_cast<uint2*>((isk ? kdst : vdst) + e) = quantize8(x, isk ? qk : qv);
+    const int32_t e = gw * (isk ? g : g - nk);
+    const uint4* src = reinterpret_cast<const uint4*>((isk ? ksrc : vsrc) + e);
+    uint8_t* dst = (isk ? kdst : vdst) + e;
+    const uint2 lo = quantize8(src[0], isk ? qk : qv);
+    if (g16) {
+      const uint2 hi = quantize8(src[1], isk ? qk : qv);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    } else {
+      *reinterpret_cast<uint2*>(dst) = lo;
+    }
   }
 }
 
@@ -376,7 +410,9 @@ cudaError_t launch_append(const CacheView& c, const uint16_t* k_new, const uint1
   a.realloc_pages = realloc_pages;
   a.n_realloc = n_realloc;
   const int64_t rows = static_cast<int64_t>(T) * c.Hkv;
-  const bool batched = c.v_pages != nullptr && c.Dk / 8 + c.Dv / 8 <= 32 &&
+  const int32_t gt = c.Dk / 16 + c.Dv / 16;   // 16-value groups per token (batched case)
+  const bool batched = c.v_pages != nullptr && c.Dk % 16 == 0 && c.Dv % 16 == 0 && gt >= 4 &&
+                       gt <= 16 && 32 % gt == 0 &&
                        (!c.fp8 || c.scale_mode != 2);
   a.batched = batched ? kRowsPerWarp : 1;
   // batched: one warp per (head, group of kRowsPerWarp tokens); else one per row
