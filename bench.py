@@ -212,32 +212,45 @@ def capture(fn, stream):
 
 
 def dist_setup(args):
+    """One process per GPU under torchrun (NCCL); without CUDA (the multi-rank
+    tests on the host) the same plumbing runs over gloo."""
     if args.gpus <= 1 and "WORLD_SIZE" not in os.environ:
         return 0, 1, 0
     import torch.distributed as dist
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                            device_id=torch.device("cuda", local))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     return rank, world, local
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (timings are taken as the slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_rank: float, ms_max: float) -> float:
+    """Whole-job throughput: every rank's bytes over the slowest rank's time."""
+    return world * bytes_per_rank / (ms_max * 1e-3) / 1e9
 
 
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 # ---------------------------------------------------------------------------
@@ -436,7 +449,7 @@ def run_ours(args):
         del g_step, g_nochk, g_dec
         bf16 = run_bf16(wl, args, stream, world, dev)
 
-    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbs(world, kv_bytes, ms_step)
     # kernels per step: append, validate, then decode (wide: query pre-pass +
     # decode + combine; otherwise decode + combine)
     launches = 2 + (3 if is_wide(s) else 2)
@@ -540,7 +553,7 @@ def run_long(args):
     # in the detailed graphs the no-check step records the same events around an
     # empty slot: its gap is the event overhead, subtracted from the validate slot
     val = mean(t_val[det & (kind == 1)]) - mean(t_val[det & (kind == 2)])
-    gbs = world * kv[plain].sum() / (max_over_ranks(float(ms[plain].sum()), world) * 1e-3) / 1e9
+    gbs = whole_job_gbs(world, kv[plain].sum(), max_over_ranks(float(ms[plain].sum()), world))
     hbm, hbm_kind = peaks()
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
@@ -626,7 +639,7 @@ def run_e2e(db, args, stream, kv_bytes, world):
         ga, gb = db.capture_io_pipelined(host_in, host_out, stream)
         ms = timed([ga.replay, gb.replay])
         del ga, gb
-    gbs = lambda m: world * kv_bytes / (m * 1e-3) / 1e9
+    gbs = lambda m: whole_job_gbs(world, kv_bytes, m)
     return {"value": gbs(ms), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "steps": K, "path": "python binding -> C ABI; two CUDA graphs in turn, each a step "
@@ -656,7 +669,7 @@ def run_bf16(wl_fp8, args, stream, world, dev):
         msd = max_over_ranks(time_graph(gd, args.steps, stream), world)
     kv = 2 * wl_fp8.kv_bytes_read()
     hbm, _ = peaks()
-    res = {"ms_per_step": ms, "kv_gbs": world * kv / (ms * 1e-3) / 1e9,
+    res = {"ms_per_step": ms, "kv_gbs": whole_job_gbs(world, kv, ms),
            "decode_ms_per_launch": msd, "decode_kv_gbs": kv / (msd * 1e-3) / 1e9,
            "decode_frac_of_hbm": kv / (msd * 1e-3) / 1e9 / hbm,
            "decode_tokens_per_s": world * wl_fp8.B / (ms * 1e-3)}
