@@ -273,9 +273,12 @@ kvq_status kvq_decode_noalloc(const kvq_cache* cache, const void* q, int32_t num
 kvq_status kvq_e4m3_encode_bits(uint32_t start, uint32_t count, uint8_t* out, void* stream);
 
 /*
- * The division kvq_append performs, exposed for exhaustive checks:
+ * The quantize step of kvq_append, exposed for exhaustive checks:
  * out[i] = E4M3(x / scale) for x the float with bit pattern start + i,
  * where x / scale is the IEEE binary32 quotient (round to nearest even).
+ * It is computed as kvq_append computes it, which reaches that quotient
+ * without a division per value where the arithmetic allows (the product
+ * by the rounded reciprocal with one FMA correction) and divides elsewhere.
  * scale must be positive and finite.  out: u8 [count].
  */
 kvq_status kvq_e4m3_quantize_bits(uint32_t start, uint32_t count, float scale, uint8_t* out,
