@@ -213,15 +213,19 @@ def test_two_tokens_closed_form():
     c = _single_page_cache(16)
     c.k_pages[1, 0, :2] = r.integers(0, 0x7E, (2, 16))
     c.v_pages[1, 0, :2] = r.integers(0, 0x7E, (2, 16))
-    qt = torch.randn(1, 1, 16).to(torch.bfloat16)
+    qt = torch.randn(1, 1, 16, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
     o, l = oracle.decode(c, bf16_bits(qt), np.array([[1]], np.int32), np.array([2], np.int32),
                          None, 1.0)
     kh = torch.from_numpy(c.k_pages[1, 0, :2]).view(torch.float8_e4m3fn).double() * 0.5
     vh = torch.from_numpy(c.v_pages[1, 0, :2]).view(torch.float8_e4m3fn).double() * 0.25
     s = (kh @ qt.double()[0, 0]).numpy()
-    w1 = 1.0 / (1.0 + math.exp(s[1] - s[0]))          # sigma(s1 - s2)
-    np.testing.assert_allclose(o[0], w1 * vh[0].numpy() + (1 - w1) * vh[1].numpy(), atol=1e-13)
-    np.testing.assert_allclose(l[0], max(s) + math.log1p(math.exp(-abs(s[0] - s[1]))), atol=1e-13)
+    d = s[1] - s[0]                                    # weight of token 0: sigma(s0 - s1)
+    w1 = 1.0 / (1.0 + math.exp(d)) if d <= 0 else math.exp(-d) / (1.0 + math.exp(-d))
+    want = w1 * vh[0].numpy() + (1 - w1) * vh[1].numpy()
+    scale = float(np.abs(vh.numpy()).max())
+    np.testing.assert_allclose(o[0], want, rtol=0, atol=1e-14 * max(1.0, scale))
+    np.testing.assert_allclose(l[0], max(s) + math.log1p(math.exp(-abs(d))),
+                               rtol=0, atol=1e-14 * max(1.0, float(np.abs(s).max())))
 
 
 def test_zero_query_gives_mean_of_values():
