@@ -27,10 +27,10 @@
 //    M=128 (64 rows per SM), N=64, K=32 E4M3 MMA uses the tensor core
 //    poorly unless several are in flight.  So two warps issue: stream k
 //    takes every other 32-dim K-step of QK^T (both query terms) into its
-//    own S accumulator, then PV of the previous block for value-dim half
-//    k (N = 256).  The softmax adds the partial scores; the fixed order per
-//    stream keeps PV, which frees the P and V buffers, from queuing behind
-//    QK^T.
+//    own S accumulator (three per stream, so QK^T runs two blocks ahead),
+//    then PV of the block two back for value-dim half k (N = 256).  The
+//    softmax adds the partial scores; the fixed order per stream keeps PV,
+//    which frees the P and V buffers, from queuing behind QK^T.
 //  * PV: kind::f16.  P goes to f16 with the token's scale folded in; V is
 //    converted from E4M3 to f16 exactly, as V * 2^-8, by moving bits on the
 //    integer pipes (the conversion unit is left to exp2 and the P packing);
@@ -42,15 +42,17 @@
 //    PV is split by value dims, so the V conversion reads the 32 tokens it
 //    lacks from the other SM's stage through distributed shared memory
 //    instead of loading them again.
-//  * Softmax: each SM's TMEM lane holds one head and 32 of the block's 64
-//    tokens (the two halves of the N range sit in lanes 0-63 and 64-127), so
-//    a head's two lanes exchange one float per block.  Scores are scaled to
-//    base 2 and exponentiated against a reference max that moves only when a
-//    score exceeds it by 2^8 (then O is rescaled in TMEM).
+//  * Softmax: eight warps per SM; each thread holds one head and 16 of the
+//    block's 64 tokens (TMEM lane quarter and column half), and the four
+//    warps holding the same 32 heads exchange partial maxima and sums
+//    through shared memory.  Scores are scaled to base 2 and exponentiated
+//    against a reference max that moves only when a score exceeds it by 2^8
+//    (then O is rescaled in TMEM).
 //  * Warp roles per CTA: 0 TMA producer (three key stages, page ids read 32
 //    blocks ahead); 1-2 MMA streams (leader CTA only; warp 1 also owns the
 //    tensor memory); 3-10 softmax, P and O read-out; 11-14 V conversion.
-//    S and converted V are double-buffered, P triple-buffered.
+//    S has three buffers per MMA stream; converted V and P two each, freed
+//    by the completion of the PV that read them.
 //  * Work split as in the 8-head kernel: the pre-pass also writes the prefix
 //    of 64-token blocks over the sequences, the blocks of all sequences are
 //    split evenly over the CTA pairs (split-KV), each pair writes one
