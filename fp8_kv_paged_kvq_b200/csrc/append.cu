@@ -60,10 +60,10 @@ __global__ void scale_from_amax_kernel(const float* __restrict__ amax, float* __
 }
 
 // ---------------------------------------------------------------------------
-// Append: one warp per (token, kv head); the last block also bumps tags.
-// The warp's lanes take the row's 8-value groups in turn across the K row
-// and then the V row (for head dims 128 that is one group per lane), so a
-// half-warp writes 128 contiguous code bytes with 8-byte stores.
+// Append: the token blocks quantize and write the new rows (a warp per
+// head and 8 tokens, or per row; see append_rows_batched and the per-row
+// path in append_kernel), lanes holding 16-value groups written with one
+// 16-byte store each; the last block bumps the tags of reallocated pages.
 // ---------------------------------------------------------------------------
 // The quotient v / s that the E4M3 encode rounds, RN(v / s), without a
 // hardware division per value.  r = RN(1/s) is worked out once per scale.

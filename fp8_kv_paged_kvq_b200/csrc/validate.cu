@@ -6,13 +6,17 @@
 // modelov Kimi a GLM kompresiou cache a váh" (aifeed.sk), section "Kvalita
 // odpovedí a integrita spoločnej cache".
 //
-// Each request gets a thread-block cluster of C <= 8 CTAs, enough that one
-// round of loads covers its block-table row: CTA r checks entries
-// r*kPerCta + k*kValThreads + tid (+ C*kPerCta per further round).  The CTAs
-// combine their flags through distributed shared memory and rank 0 writes the
-// request's mask byte, so no separate clear is needed.  The cost is launch
-// latency plus, after the sequence length, two dependent loads per entry:
-// the block-table entry with its expected tag, then the live tag.
+// Two kernels.  Batches of up to 4,096 requests run validate_flat_kernel
+// (below): one small CTA per SM over all requests' entries, sized to share
+// the SM with the decode launch that follows.  Larger batches run
+// validate_kernel: each request gets a thread-block cluster of C <= 8 CTAs,
+// enough that one round of loads covers its block-table row; CTA r checks
+// entries r*kPerCta + k*kValThreads + tid (+ C*kPerCta per further round).
+// The CTAs combine their flags through distributed shared memory and rank 0
+// writes the request's mask byte, so no separate clear is needed.  Either
+// way the cost is launch latency plus, after the sequence length, two
+// dependent loads per entry: the block-table entry with its expected tag,
+// then the live tag.
 #include <cooperative_groups.h>
 
 #include "kvq_device.cuh"
