@@ -1,7 +1,8 @@
 """Benchmark of the FP8 paged decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa|ragged|long] [--no-bf16] [--no-cpu-baseline]
+                    [--workload gqa|ragged|wide|long] [--no-bf16] [--no-cpu-baseline]
+                    [--sweep]
 
 A step is one pass of the whole hot path over one decode batch:
 kvq_append (the new token of every sequence) -> kvq_validate (page tags ->
@@ -15,6 +16,17 @@ The cache (537 MB of codes) is larger than L2, so no flush is needed.
 N independent replicas (one per GPU, no collective on the data path) and
 reports the aggregate.  `--impl reference` times the CPU oracle on a bounded
 sample of the same workload.
+
+The JSON line also carries: `roofline` (the decode call against the measured
+HBM copy bandwidth, or for the wide shape the measured bf16 tensor peak),
+`e2e` (the step through the Python API with its inputs copied from pinned
+host memory and its results read back every step, host traffic overlapped
+with the neighbouring steps; serial and eager forms beside it),
+`cpu_baseline` (the oracle on host cores), the BF16 cache on the same shape,
+the bulk prompt quantize, clocks sampled during the timed region and the
+number of kernel launches timed.  `--workload long` runs the 1,000-step loop
+with the tag check's cost; `--sweep` the FP8 / BF16 capacity and
+concurrency sweep.
 """
 from __future__ import annotations
 
