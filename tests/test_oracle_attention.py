@@ -306,3 +306,74 @@ def test_scales_independent_of_oracle(spec):
         am = a.amax() if spec.scale_mode == W.SCALE_TENSOR else a.amax(dim=(0, 2))
         want = (am / torch.tensor(448.0)).numpy().astype(np.float32).reshape(-1)
         assert np.array_equal(sc, want)
+
+
+def test_amax_ignores_nan_and_folds_into_the_running_value():
+    """Reading R18 (NaN elements do not take part in the amax) against
+    numpy's nanmax, per head and over the whole tensor, with infinities, a head
+    that is all NaN (its amax stays at the running value) and a running value
+    larger than the data (kept)."""
+    r = np.random.default_rng(21)
+    x = (r.standard_normal((50, 4, 24)) * 3).astype(np.float32)
+    x[r.random(x.shape) < 0.05] = np.nan
+    x[7, 1, 3] = -np.inf
+    x[:, 2, :] = np.nan
+    bits = torch.from_numpy(x).to(torch.bfloat16)
+    xb = bits.float().numpy()                       # the bf16 values both sides see
+    with np.errstate(all="ignore"), __import__("warnings").catch_warnings():
+        __import__("warnings").simplefilter("ignore")
+        want = np.nanmax(np.abs(xb), axis=(0, 2))
+    want = np.where(np.isnan(want), 0.0, want).astype(np.float32)
+    got = oracle.amax(bf16_bits(bits), True, np.zeros(4, np.float32))
+    assert np.array_equal(got, want) and got[1] == np.inf and got[2] == 0.0
+    run = np.array([0.0, 0.0, 5.0, 1e9], np.float32)
+    got = oracle.amax(bf16_bits(bits), True, run.copy())
+    assert np.array_equal(got, np.maximum(run, want))
+    flat = np.float32(np.nanmax(np.abs(xb)))
+    assert oracle.amax(bf16_bits(bits), False, np.zeros(1, np.float32))[0] == flat
+    # all-NaN data leaves the scale at 1 (amax 0)
+    s = oracle.scales(bf16_bits(bits[:, 2:3]), per_head=False)
+    assert s[0] == 1.0
+
+
+def test_out_of_range_page_ids_read_as_zero_rows():
+    """Reading R16: a block-table entry outside [0, P) contributes tokens whose
+    K and V are zero.  Brute force: the sequence gathered by hand from the
+    pages with torch's E4M3 decoding, explicit zero rows for the bad entries,
+    dense fp64 softmax.  Every page (page 0 included) holds nonzero codes, so
+    reading any real page in place of the zeros would fail."""
+    r = np.random.default_rng(31)
+    P, ps, H, D = 6, 4, 2, 16
+    codes = lambda: r.integers(0, 0x7E, (P, H, ps, D)).astype(np.uint8) | \
+        (r.integers(0, 2, (P, H, ps, D)).astype(np.uint8) << 7)
+    kp, vp = codes(), codes()
+    ks, vs = np.array([0.5, 0.125], np.float32), np.array([0.25, 2.0], np.float32)
+    c = oracle.Cache(oracle.FP8, oracle.SCALE_HEAD, P, ps, H, D, D, kp, vp, ks, vs,
+                     np.zeros(P, np.uint32))
+    bt = np.array([[2, P + 3, 0, -1, 5], [-4, 1, 3, 0, 0]], np.int32)
+    lens = np.array([18, 9], np.int32)
+    G = 3
+    qt = torch.randn(2, G * H, D, generator=torch.Generator().manual_seed(31)).to(torch.bfloat16)
+    sm = 0.37
+    o, l = oracle.decode(c, bf16_bits(qt), bt, lens, None, sm)
+    q = qt.double().numpy()
+    for b in range(2):
+        for h in range(G * H):
+            hk = h // G
+            kh, vh = [], []
+            for j in range(lens[b]):
+                p, off = bt[b, j // ps], j % ps
+                if 0 <= p < P:
+                    k8 = torch.from_numpy(kp[p, hk, off].copy()).view(torch.float8_e4m3fn)
+                    v8 = torch.from_numpy(vp[p, hk, off].copy()).view(torch.float8_e4m3fn)
+                    kh.append((k8.float() * float(ks[hk])).double().numpy())
+                    vh.append((v8.float() * float(vs[hk])).double().numpy())
+                else:
+                    kh.append(np.zeros(D))
+                    vh.append(np.zeros(D))
+            kh, vh = np.stack(kh), np.stack(vh)
+            s = (kh @ q[b, h]) * np.float64(np.float32(sm))
+            lse = logsumexp(s)
+            i = b * G * H + h
+            np.testing.assert_allclose(o[i], np.exp(s - lse) @ vh, rtol=0, atol=1e-11)
+            assert abs(l[i] - lse) <= 1e-11
