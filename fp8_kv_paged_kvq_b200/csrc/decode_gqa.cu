@@ -18,10 +18,12 @@
 //    leaves one partial (o, lse) in the workspace at slot c + segment, which
 //    is unique because both c and the segment index grow along the unit
 //    order.  A combine launch merges the partials of each segment.
-//  * Pipeline.  Warp 0 is the producer: one lane issues TMA tile loads
-//    (16 rows of K and of V for one page and head, 128-byte swizzle) into a
-//    ring of stages completed on mbarriers.  Warps 1..NW consume stages
-//    round-robin, each with its own online-softmax state.
+//  * Pipeline.  Every warp streams its own tiles (n = warp + NW*k of the
+//    CTA's range) through S private ring slots: lane 0 issues the TMA loads
+//    of a tile (16 rows of K and of V for one page and head, 128-byte
+//    swizzle) completed on the slot's mbarrier, and re-issues the slot as soon
+//    as the warp holds that tile's fragments in registers.  Each warp keeps
+//    its own online-softmax state; the warps' states are merged per piece.
 //  * Math.  QK^T and PV run on tensor cores (mma.m16n8k16, FP32
 //    accumulate) with the token axis as M and the 8 query heads of a group
 //    as N, so no MMA row is padding.  E4M3 codes become f16 with the hardware
@@ -33,6 +35,8 @@
 //    V's d axis (and K's, consistently with Q) is permuted per thread so
 //    that each thread reads whole 16-byte swizzled chunks with
 //    conflict-free shared loads.
+#include <mutex>
+
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 #include "kvq_decode.h"
@@ -101,36 +105,42 @@ struct GqaParams {
   int32_t num_ctas;
 };
 
-// Tokens of sequence b that decode reads (0 if aborted).
-__device__ __forceinline__ int32_t seq_tokens(const GqaParams& p, int b) {
-  if (p.abort_mask != nullptr && p.abort_mask[b]) return 0;
+// Tokens of sequence b that decode reads (0 if aborted; the abort mask is
+// consulted only when use_abort is set).
+__device__ __forceinline__ int32_t seq_tokens(const GqaParams& p, int b, bool use_abort) {
+  if (use_abort && p.abort_mask != nullptr && p.abort_mask[b]) return 0;
   int64_t n = p.seq_lens[b];
   n = n < 0 ? 0 : n;
   const int64_t cap = static_cast<int64_t>(p.max_pages) * p.c.ps;
   return static_cast<int32_t>(n > cap ? cap : n);
 }
 
-// Exclusive prefix over b of Hkv * ceil(tokens_b / 16) into pre[0..B].
-// Called by all threads of the block.
-__device__ void block_prefix_units(const GqaParams& p, int32_t* pre, int32_t* scratch) {
-  const int nthr = blockDim.x, tid = threadIdx.x;
+// Exclusive prefix over b of Hkv * ceil(tokens_b / 16) into pre[0..B]: each
+// thread sums a run of sequences, a warp scan and the warps' totals give
+// each run its start.  Called by all threads of the block; scratch holds one
+// int per warp.
+__device__ void block_prefix_units(const GqaParams& p, int32_t* pre, int32_t* scratch,
+                                   bool use_abort) {
+  const int nthr = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (p.B + nthr - 1) / nthr;
-  const int lo = tid * per, hi = min(p.B, lo + per);
+  const int lo = min(p.B, tid * per), hi = min(p.B, lo + per);
   int32_t sum = 0;
-  for (int b = lo; b < hi; ++b) sum += p.c.Hkv * ((seq_tokens(p, b) + 15) >> 4);
-  scratch[tid] = sum;
-  __syncthreads();
-  if (tid == 0) {
-    int32_t run = 0;
-    for (int t = 0; t < nthr; ++t) { const int32_t v = scratch[t]; scratch[t] = run; run += v; }
-    pre[p.B] = run;
+  for (int b = lo; b < hi; ++b) sum += p.c.Hkv * ((seq_tokens(p, b, use_abort) + 15) >> 4);
+  int32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
+  if (lane == 31) scratch[warp] = incl;
   __syncthreads();
-  int32_t run = scratch[tid];
+  int32_t run = incl - sum;
+  for (int w = 0; w < warp; ++w) run += scratch[w];
   for (int b = lo; b < hi; ++b) {
     pre[b] = run;
-    run += p.c.Hkv * ((seq_tokens(p, b) + 15) >> 4);
+    run += p.c.Hkv * ((seq_tokens(p, b, use_abort) + 15) >> 4);
   }
+  if (tid == nthr - 1) pre[p.B] = run;      // the last run ends at B
   __syncthreads();
 }
 
@@ -163,7 +173,7 @@ __device__ __forceinline__ Piece make_piece(const GqaParams& p, const int32_t* p
   pc.nt = min(tiles_b - pc.t0, u1 - u);
   pc.seg = pc.b * p.c.Hkv + pc.h;
   pc.n0 = n0;
-  pc.ntok = seq_tokens(p, pc.b);
+  pc.ntok = seq_tokens(p, pc.b, true);
   return pc;
 }
 
@@ -218,29 +228,29 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  pdl_wait();                                    // the previous kernel (validate) has finished
-  block_prefix_units(p, pre, scratch);           // includes __syncthreads
-  if (blockIdx.x == 0)
-    for (int b = threadIdx.x; b <= p.B; b += blockDim.x) p.ws_pre[b] = pre[b];
-
-  const int64_t U = pre[p.B];
-  const int32_t u0 = static_cast<int32_t>(U * blockIdx.x / p.num_ctas);
-  const int32_t u1 = static_cast<int32_t>(U * (blockIdx.x + 1) / p.num_ctas);
-  if (u0 >= u1) return;                          // no units: nothing issued, nothing to wait on
-
-  // ---------------- this warp's pipeline ----------------
-  // The CTA's tiles n = 0 .. u1-u0-1 are dealt round-robin: warp w takes
-  // n = w + NW*k, k = 0 .. kw-1, and keeps them in its own S slots
-  // (slot k % S).  When the warp has pulled tile k's fragments into
-  // registers it issues the TMA loads of tile k + S into the same slot.
-  const int cw = warp;
-  const int32_t n_cta = u1 - u0;
-  const int32_t kw = n_cta > cw ? (n_cta - cw + NW - 1) / NW : 0;
-  uint64_t* my_full = full + cw * S;
-  uint8_t* my_stage = smem + K::kOffStages + cw * S * K::kStageBytes;
-  int32_t* my_page = slot_page + cw * S;
   if (lane == 0) { tma_prefetch_desc(&k_map); tma_prefetch_desc(&v_map); }
 
+  // The work plan.  Before the dependency wait the kernel reads only what no
+  // kernel of this library writes (sequence lengths and block-table entries)
+  // and writes nothing to global memory: it lays out the units as if no
+  // request were aborted and looks up its first pages.  After the wait it
+  // reads the abort mask and redoes the plan only if some request aborted.
+  // The units go to the first N = min(num_ctas, U) CTAs, so that every
+  // working CTA has at least one (the combine relies on it).
+  const int cw = warp;
+  int64_t U = 0, N = 0;
+  int32_t u0 = 0, u1 = 0, kw = 0;
+  auto plan = [&](bool use_abort) {
+    block_prefix_units(p, pre, scratch, use_abort);  // includes __syncthreads
+    U = pre[p.B];
+    N = min(static_cast<int64_t>(p.num_ctas), U);
+    const bool works = static_cast<int64_t>(blockIdx.x) < N;
+    u0 = works ? static_cast<int32_t>(U * blockIdx.x / N) : 0;
+    u1 = works ? static_cast<int32_t>(U * (blockIdx.x + 1) / N) : 0;
+    // warp cw takes the CTA's tiles n = cw + NW*k, k = 0 .. kw-1
+    const int32_t n_cta = u1 - u0;
+    kw = n_cta > cw ? (n_cta - cw + NW - 1) / NW : 0;
+  };
   // TMA coordinates of warp-local tile k0 + lane (page id; kv head << 16 | row offset).
   auto lookup = [&](int32_t k0, int32_t& page, int32_t& hy) {
     page = 0;
@@ -258,8 +268,33 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
     }
   };
   int32_t cur_page, cur_hy, nxt_page, nxt_hy, batch0 = 0;
+  plan(false);
   lookup(0, cur_page, cur_hy);
   lookup(32, nxt_page, nxt_hy);
+
+  pdl_wait();                                    // the previous kernel (validate) has finished
+  if (p.abort_mask != nullptr) {
+    int any = 0;
+    for (int b = threadIdx.x; b < p.B; b += blockDim.x) any |= p.abort_mask[b];
+    if (__syncthreads_or(any)) {
+      plan(true);
+      lookup(0, cur_page, cur_hy);
+      lookup(32, nxt_page, nxt_hy);
+    }
+  }
+  if (blockIdx.x == 0)
+    for (int b = threadIdx.x; b <= p.B; b += blockDim.x) p.ws_pre[b] = pre[b];
+  if (u0 >= u1) return;                          // no units: nothing issued, nothing to wait on
+
+  // ---------------- this warp's pipeline ----------------
+  // The warp keeps its tiles in its own S slots (slot k % S).  When it has
+  // pulled tile k's fragments into registers it issues the TMA loads of tile
+  // k + S into the same slot.  The loads are marked evict-first in L2: the
+  // cache is streamed once per call.
+  uint64_t* my_full = full + cw * S;
+  uint8_t* my_stage = smem + K::kOffStages + cw * S * K::kStageBytes;
+  int32_t* my_page = slot_page + cw * S;
+  const uint64_t l2_stream = l2_policy_evict_first();
   int32_t issued = 0;                            // tiles of this warp issued so far
   // Issue warp-local tile `issued` (all lanes call; tiles go out in order).
   auto issue_next = [&]() {
@@ -280,10 +315,10 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
       mbar_arrive_expect_tx(&my_full[sl], K::kStageBytes);
 #pragma unroll
       for (int x = 0; x < L::kBoxes; ++x) {
-        tma_load_4d(st + x * 2048, &k_map, &my_full[sl], x * L::kBoxElems, hy & 0xFFFF, hy >> 16,
-                    page);
-        tma_load_4d(st + L::kTileBytes + x * 2048, &v_map, &my_full[sl], x * L::kBoxElems,
-                    hy & 0xFFFF, hy >> 16, page);
+        tma_load_4d_hint(st + x * 2048, &k_map, &my_full[sl], x * L::kBoxElems, hy & 0xFFFF,
+                         hy >> 16, page, l2_stream);
+        tma_load_4d_hint(st + L::kTileBytes + x * 2048, &v_map, &my_full[sl], x * L::kBoxElems,
+                         hy & 0xFFFF, hy >> 16, page, l2_stream);
       }
     }
   };
@@ -589,9 +624,14 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
 // ---------------------------------------------------------------------------
 // Log-sum-exp combine.  Grid (segment = (sequence, KV head), head chunk): a
 // block merges the partials of up to kCombHeads query heads of one segment.
-// Warp w first turns the partial lse values of its heads into normalised
-// weights w_k = exp(lse_k - M) / sum_k exp(lse_k - M) (shared memory), then
-// the block forms out = sum_k w_k * o_k with coalesced 16-byte loads.
+// The decode launch gave its units to N = min(num_ctas, U) CTAs, CTA c taking
+// [c*U/N, (c+1)*U/N), so unit u belongs to CTA ((u+1)*N - 1) / U and the
+// pieces of a segment with units [S, E) are exactly the CTAs cs..ce that own
+// S and E - 1, every one of them non-empty.  Warp w turns the partial lse
+// values of its heads into a maximum M and a sum L over any number of
+// pieces; the block then forms out = sum_k exp(lse_k - M) / L * o_k with
+// coalesced 16-byte loads, taking the pieces in chunks of kCombChunk whose
+// weights it stages in shared memory.
 // ---------------------------------------------------------------------------
 struct CombineParams {
   const int32_t* ws_pre;
@@ -604,8 +644,14 @@ struct CombineParams {
 
 constexpr int kCombThreads = 256;
 constexpr int kCombHeads = 32;        // heads per block at most
-constexpr int kMaxPieces = 64;        // partials per segment at most
+constexpr int kCombChunk = 64;        // pieces whose weights are staged at once
 constexpr int kCombOutputs = 4096;    // outputs per block (heads_per_block * Dv) at most
+constexpr int kCombPerThread = kCombOutputs / 4 / kCombThreads;   // float4 outputs per thread
+
+// CTA of a launch with N working CTAs over U units that owns unit u.
+__device__ __forceinline__ int64_t owner_cta(int64_t u, int64_t N, int64_t U) {
+  return ((u + 1) * N - 1) / U;
+}
 
 __global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const CombineParams p) {
   pdl_wait();                                    // the decode kernel has finished
@@ -624,83 +670,95 @@ __global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const Combine
       for (int hh = threadIdx.x; hh < nh; hh += blockDim.x) lse[hh] = -__int_as_float(0x7f800000);
     return;
   }
+  // U >= tiles_b > 0 here
   const int64_t S = p.ws_pre[b] + static_cast<int64_t>(h) * tiles_b, E = S + tiles_b;
-  const int64_t N = p.num_ctas;
-  __shared__ int64_t slots[kMaxPieces];
-  __shared__ int np_sh;
-  __shared__ float wts[kCombHeads][kMaxPieces];
-  if (threadIdx.x == 0) {
-    // first CTA whose range [c*U/N, (c+1)*U/N) contains unit S
-    int64_t c = S * N / U;
-    while (c + 1 < N && (c + 1) * U / N <= S) ++c;
-    while (c > 0 && c * U / N > S) --c;
-    // partial slots of the CTAs that cover part of [S, E); CTAs with an empty
-    // range (possible only when U < N) wrote nothing and are skipped
-    int np = 0;
-    for (int64_t cc = c; cc < N && cc * U / N < E; ++cc) {
-      if ((cc + 1) * U / N == cc * U / N) continue;
-      if (np < kMaxPieces) slots[np] = cc + seg;
-      ++np;
-    }
-    np_sh = np;
-  }
-  __syncthreads();
-  const int np = np_sh;
-  if (np > kMaxPieces) {
-    // more partials than the combine can hold: a launch configuration with
-    // far more CTAs than tiles per segment; flag it instead of reading past
-    if (threadIdx.x == 0) atomicOr(&g_error_flags, 2u);
-    return;
-  }
+  const int64_t N = min(static_cast<int64_t>(p.num_ctas), U);
+  const int64_t cs = owner_cta(S, N, U);
+  const int np = static_cast<int>(owner_cta(E - 1, N, U) - cs + 1);
+  const int64_t slot0 = cs + seg;               // slot of piece k: slot0 + k
+  __shared__ float m_sh[kCombHeads], inv_sh[kCombHeads];
+  __shared__ float wts[kCombHeads][kCombChunk];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float kNegInf = -__int_as_float(0x7f800000);
   for (int hh = warp; hh < nh; hh += kCombThreads / 32) {
     const int head = h0 + hh;
-    const float a0 = lane < np ? p.ws_lse[slots[lane] * p.G + head] : kNegInf;
-    const float a1 = lane + 32 < np ? p.ws_lse[slots[lane + 32] * p.G + head] : kNegInf;
-    float M = fmaxf(a0, a1);
+    const float* l = p.ws_lse + slot0 * p.G + head;   // piece k at l[k * G]
+    float M = kNegInf;
+    for (int k = lane; k < np; k += 32) M = fmaxf(M, l[static_cast<int64_t>(k) * p.G]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float e0 = lane < np ? __expf(a0 - M) : 0.0f;
-    const float e1 = lane + 32 < np ? __expf(a1 - M) : 0.0f;
-    float L = e0 + e1;
+    float L = 0.0f;
+    for (int k = lane; k < np; k += 32) L += __expf(l[static_cast<int64_t>(k) * p.G] - M);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    const float inv = 1.0f / L;
-    if (lane < np) wts[hh][lane] = e0 * inv;
-    if (lane + 32 < np) wts[hh][lane + 32] = e1 * inv;
-    if (lse && lane == 0) lse[hh] = np == 1 ? a0 : M + __logf(L);
+    if (lane == 0) {
+      m_sh[hh] = M;
+      inv_sh[hh] = 1.0f / L;
+      if (lse) lse[hh] = np == 1 ? l[0] : M + __logf(L);
+    }
   }
-  __syncthreads();
-  // outputs in groups of four consecutive dims (Dv is a multiple of 4)
+  // outputs in groups of four consecutive dims (Dv is a multiple of 4); thread
+  // t holds groups t, t + kCombThreads, ...
   const int dq = p.Dv >> 2;
-  const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
-  for (int i4 = threadIdx.x; i4 < nh * dq; i4 += blockDim.x) {
-    const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
-    const int head = h0 + hh;
-    float4 acc;
-    if (np == 1) {
-      acc = *reinterpret_cast<const float4*>(p.ws_o + (slots[0] * p.G + head) * p.Dv + d);
-    } else {
-      acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-      for (int k = 0; k < np; ++k) {
-        const float4 v = *reinterpret_cast<const float4*>(p.ws_o + (slots[k] * p.G + head) * p.Dv + d);
-        const float w = wts[hh][k];
-        acc.x += w * v.x;
-        acc.y += w * v.y;
-        acc.z += w * v.z;
-        acc.w += w * v.w;
+  const int n4 = nh * dq;
+  float4 acc[kCombPerThread];
+#pragma unroll
+  for (int r = 0; r < kCombPerThread; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (np == 1) {
+    // a single piece is copied bit for bit
+#pragma unroll
+    for (int r = 0; r < kCombPerThread; ++r) {
+      const int i4 = threadIdx.x + r * kCombThreads;
+      if (i4 < n4) {
+        const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
+        acc[r] = *reinterpret_cast<const float4*>(p.ws_o + (slot0 * p.G + h0 + hh) * p.Dv + d);
       }
     }
+  } else {
+    __syncthreads();                             // m_sh, inv_sh
+    for (int base = 0; base < np; base += kCombChunk) {
+      const int nk = min(kCombChunk, np - base);
+      for (int idx = threadIdx.x; idx < nh * nk; idx += kCombThreads) {
+        const int hh = idx / nk, k = idx - hh * nk;
+        const float a = p.ws_lse[(slot0 + base + k) * p.G + h0 + hh];
+        wts[hh][k] = __expf(a - m_sh[hh]) * inv_sh[hh];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < kCombPerThread; ++r) {
+        const int i4 = threadIdx.x + r * kCombThreads;
+        if (i4 < n4) {
+          const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
+          const float* o = p.ws_o + ((slot0 + base) * p.G + h0 + hh) * p.Dv + d;
+          const int64_t stride = static_cast<int64_t>(p.G) * p.Dv;   // next piece
+#pragma unroll 4
+          for (int k = 0; k < nk; ++k) {
+            const float4 v = *reinterpret_cast<const float4*>(o + k * stride);
+            const float w = wts[hh][k];
+            acc[r].x += w * v.x;
+            acc[r].y += w * v.y;
+            acc[r].z += w * v.z;
+            acc[r].w += w * v.w;
+          }
+        }
+      }
+      __syncthreads();                           // wts reused by the next chunk
+    }
+  }
+  const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+#pragma unroll
+  for (int r = 0; r < kCombPerThread; ++r) {
+    const int i4 = threadIdx.x + r * kCombThreads;
+    if (i4 >= n4) continue;
+    const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
     float* dst = out + hh * p.Dv + d;
     if (vec_out) {
-      *reinterpret_cast<float4*>(dst) = acc;
+      *reinterpret_cast<float4*>(dst) = acc[r];
     } else {
-      dst[0] = acc.x;
-      dst[1] = acc.y;
-      dst[2] = acc.z;
-      dst[3] = acc.w;
+      dst[0] = acc[r].x;
+      dst[1] = acc[r].y;
+      dst[2] = acc[r].z;
+      dst[3] = acc[r].w;
     }
   }
 }
@@ -726,7 +784,7 @@ cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const
   int hpb = kCombOutputs / (Dv > 0 ? Dv : 1);
   hpb = hpb < 1 ? 1 : (hpb > kCombHeads ? kCombHeads : hpb);
   cp.heads_per_block = hpb;
-  if (Dv % 4 != 0) return cudaErrorInvalidValue;
+  if (Dv % 4 != 0 || Dv > kCombOutputs) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(B * Hkv), static_cast<unsigned>((G + hpb - 1) / hpb));
   if (B * Hkv == 0) return cudaSuccess;
   return launch_pdl(lse_combine_kernel, grid, dim3(kCombThreads), 0, stream, cp);
@@ -737,8 +795,10 @@ cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const
 template <bool FP8, int D, int NT, int NW, int NS>
 static cudaError_t prepare_gqa(int dev) {
   using K = GqaKernel<FP8, D, NT, NW, NS>;
+  static std::mutex mu;
   static bool done[64] = {};
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
   if (done[dev]) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(gqa_decode_kernel<FP8, D, NT, NW, NS>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -797,15 +857,20 @@ static int gqa_blocks_per_sm(int dev, int B) {
   using C = GqaConfig<FP8, D, NT>;
   using K = GqaKernel<FP8, D, NT, C::kNW, C::kNS>;
   // cache the last query per device: the answer depends only on B here
+  static std::mutex mu;
   static int last_b[64], last_n[64];
   static bool have[64] = {};
   if (dev < 0 || dev >= 64) return 0;
-  if (have[dev] && last_b[dev] == B) return last_n[dev];
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (have[dev] && last_b[dev] == B) return last_n[dev];
+  }
   if (prepare_gqa<FP8, D, NT, C::kNW, C::kNS>(dev) != cudaSuccess) return 0;
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gqa_decode_kernel<FP8, D, NT, C::kNW, C::kNS>,
                                                     K::kThreads, K::smem_bytes(B)) != cudaSuccess)
     return 0;
+  std::lock_guard<std::mutex> lock(mu);
   last_b[dev] = B;
   last_n[dev] = n;
   have[dev] = true;

@@ -58,6 +58,8 @@
 //    split evenly over the CTA pairs (split-KV), each pair writes one
 //    partial (o, lse) per sequence piece at slot pair + sequence, and the
 //    log-sum-exp combine merges them.
+#include <mutex>
+
 #include "kvq_decode.h"
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
@@ -176,28 +178,29 @@ __global__ void __launch_bounds__(kPrepThreads) wide_prep_kernel(const Params p)
   pdl_wait();                                    // the previous kernel (validate) has finished
   const int tid = threadIdx.x;
   if (blockIdx.x == 2 * p.B) {
-    __shared__ int32_t scratch[kPrepThreads];
+    // each thread sums a run of sequences; a warp scan and the warps' totals
+    // give each run its start
+    __shared__ int32_t warp_tot[kPrepThreads / 32];
+    const int lane = tid & 31, warp = tid >> 5;
     const int per = (p.B + kPrepThreads - 1) / kPrepThreads;
-    const int lo = tid * per, hi = min(p.B, lo + per);
+    const int lo = min(p.B, tid * per), hi = min(p.B, lo + per);
     int32_t sum = 0;
     for (int b = lo; b < hi; ++b) sum += (seq_tokens(p, b) + kBlk - 1) / kBlk;
-    scratch[tid] = sum;
-    __syncthreads();
-    if (tid == 0) {
-      int32_t run = 0;
-      for (int t = 0; t < kPrepThreads; ++t) {
-        const int32_t v = scratch[t];
-        scratch[t] = run;
-        run += v;
-      }
-      p.ws_pre[p.B] = run;
+    int32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
+    if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
-    int32_t run = scratch[tid];
+    int32_t run = incl - sum;
+    for (int w = 0; w < warp; ++w) run += warp_tot[w];
     for (int b = lo; b < hi; ++b) {
       p.ws_pre[b] = run;
       run += (seq_tokens(p, b) + kBlk - 1) / kBlk;
     }
+    if (tid == kPrepThreads - 1) p.ws_pre[p.B] = run;   // the last run ends at B
     return;
   }
   const int b = blockIdx.x >> 1, r = blockIdx.x & 1;
@@ -375,9 +378,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();                                 // the combine may launch (it waits for us)
   pdl_wait();                                    // the pre-pass has finished
 
+  // The blocks go to the first N = min(num_pairs, U) pairs, so that every
+  // working pair has at least one (the combine relies on it); the others
+  // get an empty range and only set up and tear down.
   const int64_t U = __ldg(p.ws_pre + p.B);
-  const int32_t u0 = static_cast<int32_t>(U * pair / p.num_pairs);
-  const int32_t u1 = static_cast<int32_t>(U * (pair + 1) / p.num_pairs);
+  const int64_t N = min(static_cast<int64_t>(p.num_pairs), U);
+  const bool works = pair < N;
+  const int32_t u0 = works ? static_cast<int32_t>(U * pair / N) : 0;
+  const int32_t u1 = works ? static_cast<int32_t>(U * (pair + 1) / N) : 0;
   const int32_t nblk = u1 - u0;
 
   if (warp == 0) {
@@ -799,8 +807,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Host side
 // ---------------------------------------------------------------------------
 static cudaError_t prepare_wide(int dev) {
+  static std::mutex mu;
   static bool done[64] = {};
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
   if (done[dev]) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(wide::wide_decode_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -813,10 +823,14 @@ int wide_default_pairs(int B) {
   (void)B;   // the wide kernel's shared memory does not depend on the batch size
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static std::mutex mu;
   static int last_n[64];
   static bool have[64] = {};
   if (dev < 0 || dev >= 64) return 0;
-  if (have[dev]) return last_n[dev];
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (have[dev]) return last_n[dev];
+  }
   if (prepare_wide(dev) != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2);
@@ -831,6 +845,7 @@ int wide_default_pairs(int B) {
   cfg.numAttrs = 1;
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, wide::wide_decode_kernel, &cfg) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
   last_n[dev] = n;
   have[dev] = true;
   return n;

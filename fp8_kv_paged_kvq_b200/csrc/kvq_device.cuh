@@ -11,9 +11,8 @@
 
 namespace kvq {
 
-// Library-wide device error word (bit 0: a bounded wait gave up; bit 1: a
-// combine found more partials than it can hold).  libkvq is one translation
-// unit, so this definition appears once.
+// Library-wide device error word (bit 0: a bounded wait gave up).  libkvq is
+// one translation unit, so this definition appears once.
 __device__ uint32_t g_error_flags = 0;
 constexpr uint32_t kErrWaitTimeout = 1u;
 
@@ -114,6 +113,42 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
       "r"(c3)
       : "memory");
+}
+
+// L2 eviction policies (createpolicy): streamed data that is read once per
+// call is marked evict-first, so that the small tables the next call reads
+// again (page tags, block tables, expected tags) stay in L2 between calls.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// tma_load_4d with an L2 eviction policy for the loaded lines.
+__device__ __forceinline__ void tma_load_4d_hint(void* smem_dst, const CUtensorMap* map,
+                                                 uint64_t* bar, int32_t c0, int32_t c1,
+                                                 int32_t c2, int32_t c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+      "r"(c3), "l"(policy)
+      : "memory");
+}
+
+// 32-bit global load with an L2 eviction policy.
+__device__ __forceinline__ uint32_t ld_global_hint(const void* p, uint64_t policy) {
+  uint32_t v;
+  asm volatile("ld.global.L2::cache_hint.b32 %0, [%1], %2;"
+               : "=r"(v)
+               : "l"(reinterpret_cast<uint64_t>(p)), "l"(policy)
+               : "memory");
+  return v;
 }
 
 // ---------------------------------------------------------------------------

@@ -19,6 +19,8 @@
 // then the live tag.
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
@@ -186,6 +188,10 @@ __global__ void __maxnreg__(32)
     b = lo;
     i = f - pre[lo];
   };
+  // The entries, expected tags and live tags are read with an evict-last L2
+  // policy: they are a few hundred KB that every step reads again, next to a
+  // decode launch that streams the whole cache through L2 (evict-first).
+  const uint64_t keep = l2_policy_evict_last();
   int32_t page[kFlatPer];
   uint32_t want[kFlatPer];
   auto load_round = [&](int32_t r) {
@@ -198,8 +204,8 @@ __global__ void __maxnreg__(32)
       if (f < f1) {
         locate(f, b, b, i);                 // entries grow with k: start from the last
         const int64_t e = static_cast<int64_t>(b) * max_pages + i;
-        page[k] = block_table[e];
-        want[k] = expected[e];
+        page[k] = static_cast<int32_t>(ld_global_hint(block_table + e, keep));
+        want[k] = ld_global_hint(expected + e, keep);
       }
     }
   };
@@ -222,7 +228,7 @@ __global__ void __maxnreg__(32)
       const int32_t f = r + k * kFlatThreads + tid;
       const int32_t p = page[k];
       const bool in = p >= 0 && p < P;
-      const uint32_t live = in ? tags[in ? p : 0] : 0u;
+      const uint32_t live = in ? ld_global_hint(tags + p, keep) : 0u;
       if (f < f1 && (!in || live != want[k])) bits |= 1u << k;
     }
     if (bits != 0) {
@@ -277,25 +283,34 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
     return cudaMemsetAsync(n_aborted, 0, sizeof(int32_t), stream);
   }
   if (B <= kFlatMaxB && static_cast<int64_t>(B) * max_pages <= 0x7fffffff) {
-    static int sms[64] = {0};
+    static std::mutex mu;
+    static int sms_of[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (sms[dev] == 0) {
-      e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
-      if (e != cudaSuccess) return e;
-      // keep the SM's shared memory at its largest split while this runs,
-      // so the decode CTAs (about 100 KB each) fit beside it
-      e = cudaFuncSetAttribute(validate_flat_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                               cudaSharedmemCarveoutMaxShared);
-      if (e != cudaSuccess) return e;
+    int sms = 0;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      if (sms_of[dev] == 0) {
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        // keep the SM's shared memory at its largest split while this runs,
+        // so the decode CTAs (about 100 KB each) fit beside it
+        e = cudaFuncSetAttribute(validate_flat_kernel,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        sms_of[dev] = n;
+      }
+      sms = sms_of[dev];
     }
     // at most one CTA per SM, and no more than B * max_pages entries need:
     // one round of kFlatPer loads per thread either way up to 148K entries
     const int64_t per_cta = static_cast<int64_t>(kFlatThreads) * kFlatPer;
     const int64_t want = (static_cast<int64_t>(B) * max_pages + per_cta - 1) / per_cta;
-    const int grid = static_cast<int>(want < 1 ? 1 : (want < sms[dev] ? want : sms[dev]));
+    const int grid = static_cast<int>(want < 1 ? 1 : (want < sms ? want : sms));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kFlatThreads);

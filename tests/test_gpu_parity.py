@@ -428,3 +428,43 @@ def test_append_every_bf16_pattern(mode):
     assert np.array_equal(c.v_pages.cpu().numpy(), oc.v_pages)
     assert np.array_equal(c.k_scale.cpu().numpy().view(np.uint32), oc.k_scale.view(np.uint32))
     assert np.array_equal(c.v_scale.cpu().numpy().view(np.uint32), oc.v_scale.view(np.uint32))
+
+
+@pytest.mark.parametrize("num_ctas", [0, 1000])
+def test_single_long_sequence_split_into_many_pieces(num_ctas):
+    """One sequence on one KV head: every 16-token tile can become its own
+    piece (256 pieces at 4,096 tokens with the default CTA count), so the
+    combine merges far more than one warp's worth of partials per head."""
+    spec = W.Spec("one_long", [4096], 16, 8, 1, 128, 128, outlier_p=0.01)
+    wl, db, oc = build_both(spec, seed=16, num_ctas=num_ctas)
+    out, lse = db.step(check_tags=False)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), "one long")
+    assert kvq.device_error() == 0
+
+
+def test_few_kv_heads_long_context_bf16_and_group_16():
+    """B = 1 with four KV heads (about 74 pieces per segment at the default
+    CTA count) on the BF16 cache, and a 16-head group on the FP8 cache."""
+    for spec in (W.Spec("b1_bf16", [4096], 16, 32, 4, 128, 128, kv_dtype=W.BF16),
+                 W.Spec("b1_g16", [3000], 16, 16, 1, 64, 64)):
+        wl, db, oc = build_both(spec, seed=17)
+        out, lse = db.step(check_tags=False)
+        torch.cuda.synchronize()
+        ro, rl = OS.decode(wl, oc)
+        assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), spec.name)
+    assert kvq.device_error() == 0
+
+
+def test_wide_single_long_sequence_many_pieces():
+    """The tensor-core path with one 8,192-token sequence: 128 blocks of 64
+    tokens over the default CTA pairs, one piece per pair."""
+    spec = W.Spec("wide_one_long", [8192], 64, 128, 1, 576, 512, v_alias=True,
+                  scale_mode=W.SCALE_TOKEN)
+    wl, db, oc = build_both(spec, seed=18)
+    out, lse = db.step(check_tags=False)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), "wide one long")
+    assert kvq.device_error() == 0

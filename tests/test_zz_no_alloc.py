@@ -42,9 +42,9 @@ def _close(a, b):
         assert (d[big] / np.abs(fb[big])).max() <= RTOL
 
 
-def _batch(spec, seed):
+def _batch(spec, seed, num_ctas=0):
     wl = W.make_workload(spec, seed=seed, device="cuda")
-    db = DecodeBatch(wl)
+    db = DecodeBatch(wl, num_ctas=num_ctas)
     db.prefill()
     db.append_new()
     db.validate()
@@ -52,7 +52,7 @@ def _batch(spec, seed):
     return db, ref_out, ref_lse
 
 
-def _noalloc(db):
+def _noalloc(db, num_ctas=0):
     out = torch.full_like(db.out, float("nan"))
     lse = torch.full_like(db.lse, float("nan"))
     st = kvq.lib().kvq_decode_noalloc(
@@ -60,7 +60,7 @@ def _noalloc(db):
         ctypes.c_void_p(db.block_table.data_ptr()), db.block_table.shape[1],
         ctypes.c_void_p(db.seq_lens.data_ptr()), db.q.shape[0],
         ctypes.c_void_p(db.abort.data_ptr()), ctypes.c_float(db.wl.sm_scale),
-        ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), 0,
+        ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(lse.data_ptr()), num_ctas,
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == kvq.KVQ_OK, kvq.lib().kvq_status_string(st)
     return out, lse
@@ -87,6 +87,32 @@ def test_noalloc_matches_allocating_decode_on_two_calls_in_a_row():
     torch.cuda.synchronize()
     _close(a2_out, ra_out)
     _close(a2_lse, ra_lse)
+    assert kvq.device_error() == 0
+
+
+def test_noalloc_wide_group_matches_allocating_decode_on_two_calls_in_a_row():
+    """The same check on the tensor-core shape (128 query heads on one KV
+    head, K 576 / V the first 512 dims, per-token scales), whose workspace also
+    holds the query images: two calls in a row on two batches.  Its partial
+    outputs take 256 KB per CTA pair, so the batch runs on 8 pairs to fit
+    the fixed array (the default pair count would be refused)."""
+    pairs = 8
+    spec_a = W.Spec("na_wide_a", [700, 65], 64, 128, 1, 576, 512, v_alias=True,
+                    scale_mode=W.SCALE_TOKEN, n_stale=1)
+    spec_b = W.Spec("na_wide_b", [1, 300, 129], 64, 128, 1, 576, 512, v_alias=True,
+                    scale_mode=W.SCALE_TOKEN)
+    db_a, ra_out, ra_lse = _batch(spec_a, seed=23, num_ctas=pairs)
+    db_b, rb_out, rb_lse = _batch(spec_b, seed=24, num_ctas=pairs)
+    assert kvq.decode_workspace_size(db_a.cache, 3, 128, pairs) <= (8 << 20)
+    torch.cuda.synchronize()
+    a_out, a_lse = _noalloc(db_a, pairs)
+    b_out, b_lse = _noalloc(db_b, pairs)
+    torch.cuda.synchronize()
+    _close(a_out, ra_out)
+    _close(a_lse, ra_lse)
+    _close(b_out, rb_out)
+    _close(b_lse, rb_lse)
+    assert torch.equal(a_out, ra_out) and torch.equal(b_out, rb_out)
     assert kvq.device_error() == 0
 
 
