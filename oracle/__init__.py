@@ -53,6 +53,11 @@ def lib():
     return _lib
 
 
+def set_threads(n: int = 0) -> int:
+    """Threads the oracle's parallel loops use (n <= 0: leave as is); returns the setting."""
+    return int(lib().oracle_set_threads(ctypes.c_int(n)))
+
+
 def _p(a):
     if a is None:
         return None

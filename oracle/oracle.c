@@ -39,9 +39,18 @@
  *   tags     u32 [P]
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+
+/* Threads the parallel loops below may use (the CPU baseline is timed on all
+ * host cores and on one).  n <= 0 keeps the current setting.  Returns the
+ * setting in force. */
+int oracle_set_threads(int n) {
+  if (n > 0) omp_set_num_threads(n);
+  return omp_get_max_threads();
+}
 
 #define ORACLE_FP8 0
 #define ORACLE_BF16 1
