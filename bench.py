@@ -1,39 +1,47 @@
-"""Benchmark of the FP8 paged decode step on B200.
+"""Benchmark of the FP8 paged decode path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa|ragged|wide|long] [--no-bf16] [--no-cpu-baseline]
-                    [--sweep]
+                    [--workload long|gqa|ragged|wide] [--no-extra] [--no-bf16]
+                    [--no-cpu-baseline] [--sweep]
 
-A step is one pass of the whole hot path over one decode batch:
-kvq_append (the new token of every sequence) -> kvq_validate (page tags ->
-abort mask) -> kvq_decode (split-KV attention + log-sum-exp combine).  The
-default workload is the GQA decode batch: 32 sequences x 8,192 tokens, page
-16, 64 query / 8 KV heads, head_dim 128, E4M3 cache with per-head scales.
-The cache (537 MB of codes) is larger than L2, so no flush is needed.
+A decode step is one pass of the whole hot path over one batch:
+kvq_append (the new token of every sequence, with tag bumps for reallocated
+pages) -> kvq_validate (page tags -> abort mask) -> kvq_decode (split-KV
+attention + log-sum-exp combine).
 
-`value` is KV GB/s: cache bytes one decode step reads / device time per step
-(CUDA events, steps replayed from a CUDA graph, max over ranks).  N > 1 runs
-N independent replicas (one per GPU, no collective on the data path) and
-reports the aggregate.  `--impl reference` times the CPU oracle on a bounded
-sample of the same workload.
+Default workload (the long-context one): 4 sequences of 262,144 tokens and 60
+of 8,192, page 16, 64 query / 8 KV heads, head_dim 128, E4M3 cache with
+per-head scales, decoded for 1,000 steps that each append a token per
+sequence (pages that fill up are replaced by reallocated pages whose tags the
+append bumps).  Steps cycle through three kinds: the tag check with 0.01% of
+the expected tags made stale (those requests abort), the tag check with
+every tag right ("clean"), and no check.  For this workload --steps and
+--warmup count passes over the 1,000-step loop; every pass repeats the same
+tag history.
 
-The JSON line also carries: `roofline` (the decode call against the measured
-HBM copy bandwidth, or for the wide shape the measured bf16 tensor peak),
-`e2e` (the step through the Python API with its inputs copied from pinned
-host memory and its results read back every step, host traffic overlapped
-with the neighbouring steps; serial and eager forms beside it),
-`cpu_baseline` (the oracle on host cores), the BF16 cache on the same shape,
-the bulk prompt quantize, clocks sampled during the timed region and the
-number of kernel launches timed.  `--workload long` runs the 1,000-step loop
-with the tag check's cost; `--sweep` the FP8 / BF16 capacity and
-concurrency sweep.
+`value` is KV GB/s on the clean steps (cache bytes a step reads / its device
+time, CUDA events around each step), `ms_per_step` their mean, and the tag
+check's cost compares the clean steps with the unchecked ones (mean and
+p95).  `roofline` is the decode call (decode kernel + combine, timed between
+events inside the steps) against the measured HBM copy bandwidth.  `e2e` is
+the loop through the Python API with every step's inputs copied from pinned
+host memory and its results read back.  `cpu_baseline` is the CPU oracle on
+a sample of the same workload, on all host cores and on one.  The line also
+carries the other decode batches (`configs`): the GQA batch (32 x 8,192), the
+ragged batch (64 sequences of 1k-32k tokens, FP8 and BF16 caches) and the
+wide-group batch (128 query heads on one KV head, 576/512 dims, tensor
+cores), each with its own step statistics and roofline.
+
+N > 1 runs N independent replicas (one per GPU, no collective on the data
+path) and reports the aggregate.  `--impl reference` times the CPU oracle on
+a bounded sample of the workload.  `--sweep` runs the FP8 / BF16 capacity
+and concurrency sweep instead.
 """
 from __future__ import annotations
 
 import argparse
 import datetime
 import json
-import math
 import os
 import statistics
 import sys
@@ -49,26 +57,31 @@ sys.path.insert(0, ROOT)
 METRIC = "FP8 paged decode attention: KV GB/s (% of HBM peak) and decode tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+DTYPE = "f16 mma / f32 accumulate (e4m3 cache)"
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="gqa")
+    ap.add_argument("--workload", default="long")
     ap.add_argument("--num-ctas", type=int, default=0)
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-extra", action="store_true",
+                    help="only the headline workload, not the other decode batches")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--loop-steps", type=int, default=1000,
                     help="decode steps of the long workload's loop")
+    ap.add_argument("--min-seconds", type=float, default=0.5,
+                    help="least device time of each timed single-batch measurement")
     ap.add_argument("--sweep", action="store_true",
                     help="capacity and concurrency sweep (FP8 vs BF16 at B = 1..64) instead of the bench line")
     ap.add_argument("--seqs", type=int, default=0,
                     help="keep only the first N sequences (smaller case for profiling)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def measured_traffic(workload, seqs):
@@ -90,21 +103,26 @@ def measured_traffic(workload, seqs):
     return None
 
 
-def peaks():
+def _peaks_file():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
-            d = json.load(f)
+            return json.load(f)
+    return None
+
+
+def peaks():
+    d = _peaks_file()
+    if d:
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
 
 
 def tensor_peak():
     """Dense bf16 TFLOP/s of this GPU (burst: the decode launch is timed on its own)."""
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            return float(json.load(f)["bf16_tflops"]), "measured"
+    d = _peaks_file()
+    if d:
+        return float(d["bf16_tflops"]), "measured"
     return FALLBACK_BF16_TFLOPS, "fallback"
 
 
@@ -113,14 +131,31 @@ def is_wide(spec) -> bool:
     return spec.num_q_heads // spec.num_kv_heads >= 64
 
 
-def decode_roofline(spec, wl, alg_bytes, ms_dec, traffic):
+def decode_alg_bytes(spec, seq_lens):
+    """Algorithmic bytes of one kvq_decode call: the cache bytes the rows read
+    (codes, + per-token scales in TOKEN mode), the query, the block-table
+    entries, out and lse."""
+    s = spec
+    lens = np.minimum(np.asarray(seq_lens, np.int64), 1 << 40)
+    el = 1 if s.kv_dtype == "fp8" else 2
+    row = el * (s.head_dim_k + (0 if s.v_alias else s.head_dim_v))
+    if s.scale_mode == "token" and s.kv_dtype == "fp8":
+        row += 4
+    kv = int(lens.sum()) * s.num_kv_heads * row
+    return (kv + s.B * s.num_q_heads * s.head_dim_k * 2
+            + int(np.ceil(lens / s.page_size).sum()) * 4
+            + s.B * s.num_q_heads * (s.head_dim_v + 1) * 4)
+
+
+def decode_roofline(spec, seq_lens, ms_dec, traffic, alg_bytes=None):
     """Roofline of one kvq_decode launch.  The 8-head kernel moves bytes
     (bound: HBM).  The wide kernel is a pair of dense contractions per token,
     QK^T (a bf16 query against keys that are exact in f16) and PV (f16), so it
     is bound by the tensor cores at the f16/bf16 rate: 2 * Hq * (Dk + Dv) FLOPs
     per decoded token."""
+    alg = decode_alg_bytes(spec, seq_lens) if alg_bytes is None else alg_bytes
     if is_wide(spec):
-        tokens = int(np.minimum(wl.seq_lens, wl.max_pages * spec.page_size).sum())
+        tokens = int(np.asarray(seq_lens, np.int64).sum())
         flops = 2.0 * spec.num_q_heads * (spec.head_dim_k + spec.head_dim_v) * tokens
         peak, kind = tensor_peak()
         achieved = flops / (ms_dec * 1e-3) / 1e12
@@ -128,14 +163,21 @@ def decode_roofline(spec, wl, alg_bytes, ms_dec, traffic):
                 "kernel": "kvq_decode (wide_prep_kernel + wide_decode_kernel + lse_combine_kernel)",
                 "achieved": achieved, "peak": peak, "peak_kind": kind + " (bf16 burst)",
                 "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": alg_bytes,
+                "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": alg,
+                "hbm_frac": alg / (ms_dec * 1e-3) / 1e9 / peaks()[0],
                 "ms_per_launch": ms_dec}
     hbm, kind = peaks()
-    achieved = alg_bytes / (ms_dec * 1e-3) / 1e9
+    achieved = alg / (ms_dec * 1e-3) / 1e9
     return {"bound": "hbm", "kernel": "kvq_decode (gqa_decode_kernel + lse_combine_kernel)",
             "achieved": achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": traffic,
-            "algorithmic_bytes_per_launch": alg_bytes, "ms_per_launch": ms_dec}
+            "algorithmic_bytes_per_launch": alg, "ms_per_launch": ms_dec}
+
+
+def stats(ms):
+    ms = np.asarray(ms, np.float64)
+    return {"mean": float(ms.mean()), "min": float(ms.min()), "median": float(np.median(ms)),
+            "p95": float(np.percentile(ms, 95)), "n": int(ms.size)}
 
 
 # ---------------------------------------------------------------------------
@@ -204,16 +246,20 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # timing helpers
 # ---------------------------------------------------------------------------
-def time_graph(graph, K, stream):
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+def time_replays(replay, stream, min_s, min_n=20, chunk=64):
+    """Per-call device times (ms) of `replay`, with CUDA events on `stream`
+    around every call, repeated until at least min_n calls and min_s seconds."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(chunk + 1)]
+    times = []
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(K):
-        graph.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / K
+    while len(times) < min_n or sum(times) < min_s * 1e3:
+        ev[0].record(stream)
+        for j in range(chunk):
+            replay()
+            ev[j + 1].record(stream)
+        torch.cuda.synchronize()
+        times += [ev[j].elapsed_time(ev[j + 1]) for j in range(chunk)]
+    return np.array(times)
 
 
 def capture(fn, stream):
@@ -329,12 +375,12 @@ def oracle_sample(spec_name, n_groups, seed=0):
     return step, kv, desc
 
 
-def cpu_baseline(spec_name, budget_s, seed=0):
-    """The oracle as it stands, timed on the host cores on a sample of the
-    workload sized to about budget_s seconds (one step)."""
+def _oracle_rate(spec_name, budget_s, threads, seed=0):
+    import oracle
     from fp8_kv_paged_kvq_b200 import workloads as W
     full = W.spec_by_name(spec_name, seed)
-    step1, _, _ = oracle_sample(spec_name, 1, seed)
+    used = oracle.set_threads(threads)
+    step1, kv1, _ = oracle_sample(spec_name, 1, seed)
     t0 = time.perf_counter()
     step1()
     t1 = time.perf_counter() - t0
@@ -343,8 +389,21 @@ def cpu_baseline(spec_name, budget_s, seed=0):
     t0 = time.perf_counter()
     step()
     dt = time.perf_counter() - t0
-    return {"value": kv / dt / 1e9, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
-            "kind": "oracle", "sample": desc, "seconds": dt}
+    return {"value": kv / dt / 1e9, "unit": "GB/s", "cores": used, "kind": "oracle",
+            "sample": desc, "seconds": dt}
+
+
+def cpu_baseline(spec_name, budget_s, seed=0):
+    """The oracle as it stands, timed on the host's cores (all, then one) on a
+    sample of the workload sized to about budget_s seconds (one step)."""
+    import oracle
+    oracle.build()
+    allc = len(os.sched_getaffinity(0))
+    res = _oracle_rate(spec_name, budget_s, allc, seed)
+    one = _oracle_rate(spec_name, budget_s / 2, 1, seed)
+    oracle.set_threads(allc)
+    res["one_core"] = one
+    return res
 
 
 # ---------------------------------------------------------------------------
@@ -398,22 +457,16 @@ def workload_desc(name, seqs=0):
 
 
 # ---------------------------------------------------------------------------
-# our arm
+# one decode batch (gqa, ragged, wide): the step, the decode call, e2e
 # ---------------------------------------------------------------------------
-def run_ours(args):
-    rank, world, local = dist_setup(args)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    import fp8_kv_paged_kvq_b200 as kvq
-    from fp8_kv_paged_kvq_b200 import build as kvq_build
+def measure_batch(name, args, dev, stream, world, e2e=True, bf16=True, cpu=True):
+    """Step and decode-call statistics of one decode batch.  The step
+    (append -> validate -> decode) and the decode call are CUDA graphs, each
+    replayed with events around every replay until args.min_seconds of device
+    time; the inputs exceed L2, so no flush is needed between replays."""
     from fp8_kv_paged_kvq_b200 import workloads as W
     from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch
-    if rank == 0:
-        kvq_build.build()
-    barrier(world) if world > 1 else None
-    kvq.lib()
-
-    spec = W.spec_by_name(args.workload)
+    spec = W.spec_by_name(name)
     if args.seqs:
         spec.seq_lens = list(spec.seq_lens)[: args.seqs]
     wl = W.make_workload(spec, seed=0, device=dev)
@@ -422,14 +475,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     kv_bytes = wl.kv_bytes_read()
     s = spec
-    alg_bytes = (kv_bytes + s.B * s.num_q_heads * s.head_dim_k * 2          # q
-                 + int(np.ceil(wl.seq_lens / s.page_size).sum()) * 4        # block table
-                 + s.B * s.num_q_heads * (s.head_dim_v + 1) * 4)            # out + lse
-    stream = torch.cuda.Stream(device=dev)
-    hbm, hbm_kind = peaks()
-
     with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
+        for _ in range(3):
             db.step(check_tags=True, stream=stream)
         torch.cuda.synchronize()
         g_step = capture(lambda: db.step(check_tags=True, stream=stream), stream)
@@ -438,229 +485,75 @@ def run_ours(args):
         for g in (g_step, g_nochk, g_dec):
             for _ in range(3):
                 g.replay()
-        torch.cuda.synchronize()
-
-        # ---- the timed region: K steps ----
         barrier(world)
-        sampler = ClockSampler(local)
-        with sampler:
-            ms_step = time_graph(g_step, args.steps, stream)
-        barrier(world)
-        ms_step = max_over_ranks(ms_step, world)
-        # dominant kernel (kvq_decode: split-KV kernel + combine), same data
-        ms_dec = max_over_ranks(time_graph(g_dec, args.steps, stream), world)
-        ms_nochk = max_over_ranks(time_graph(g_nochk, args.steps, stream), world)
-    assert kvq.device_error() == 0, "device-side wait timed out"
-
-    # ---- e2e through the public API with host buffers ----
-    e2e = run_e2e(db, args, stream, kv_bytes, world)
-
-    # ---- BF16 cache, same shapes ----
-    bf16 = None
-    if not args.no_bf16 and s.kv_dtype == W.FP8 and not s.v_alias:
-        del g_step, g_nochk, g_dec
-        bf16 = run_bf16(wl, args, stream, world, dev)
-
-    value = whole_job_gbs(world, kv_bytes, ms_step)
-    # kernels per step: append, validate, then decode (wide: query pre-pass +
-    # decode + combine; otherwise decode + combine)
-    launches = 2 + (3 if is_wide(s) else 2)
-    line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16 mma / f32 accumulate (e4m3 cache)",
-        "data": "synthetic",
-        "config": {"workload": workload_desc(args.workload, args.seqs),
-                   "step": "kvq_append + kvq_validate + kvq_decode (split-KV + LSE combine)",
-                   "l2": f"inputs exceed L2: {kv_bytes / 1e6:.0f} MB of cache read per step",
-                   "timing": "CUDA graph replay, CUDA events, max over ranks",
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
-        "decode_tokens_per_s": world * s.B / (ms_step * 1e-3),
-        "hbm_frac_of_step": value / world / hbm,
-        "validate_overhead_pct": 100.0 * (ms_step - ms_nochk) / ms_nochk,
-        "ms_per_step_without_validation": ms_nochk,
-        "roofline": decode_roofline(s, wl, alg_bytes, ms_dec,
-                                    measured_traffic(args.workload, args.seqs)),
-        "gpu_launches": launches * args.steps,
-        "clocks": sampler.summary(),
-        "e2e": e2e,
-    }
-    if bf16:
-        line["bf16_same_shape"] = bf16
-        line["fp8_vs_bf16_step_time"] = ms_step / bf16["ms_per_step"]
-    if not is_wide(s) and s.kv_dtype == W.FP8 and not args.seqs:
-        line["bulk_append"] = run_bulk_append(s, dev, stream)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=10.0)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+        t_step = time_replays(g_step.replay, stream, args.min_seconds)
+        t_nochk = time_replays(g_nochk.replay, stream, args.min_seconds)
+        t_dec = time_replays(g_dec.replay, stream, args.min_seconds)
+    st, sn, sd = stats(t_step), stats(t_nochk), stats(t_dec)
+    ms_step = max_over_ranks(st["mean"], world)
+    hbm, _ = peaks()
+    lens = np.minimum(wl.seq_lens, wl.max_pages * s.page_size)
+    res = {"workload": workload_desc(name, args.seqs),
+           "kv_bytes_per_step": kv_bytes,
+           "kv_gbs": whole_job_gbs(world, kv_bytes, ms_step),
+           "hbm_frac_of_step": kv_bytes / (ms_step * 1e-3) / 1e9 / hbm,
+           "decode_tokens_per_s": world * s.B / (ms_step * 1e-3),
+           "ms_per_step": st, "ms_per_step_without_validation": sn, "ms_decode_call": sd,
+           "validate_overhead_pct": 100.0 * (st["mean"] - sn["mean"]) / sn["mean"],
+           "roofline": decode_roofline(s, lens, max_over_ranks(sd["mean"], world),
+                                       measured_traffic(name, args.seqs)),
+           "timing": "CUDA graph replays, events around every replay, "
+                     f">= {args.min_seconds} s each; inputs exceed L2"}
+    assert_no_device_error()
+    if e2e:
+        res["e2e"] = run_e2e(db, args, stream, kv_bytes, world)
+    del g_step, g_nochk, g_dec
+    if bf16 and not args.no_bf16 and s.kv_dtype == W.FP8 and not s.v_alias:
+        res["bf16_same_shape"] = run_bf16(wl, args, stream, world, dev)
+        res["fp8_vs_bf16_step_time"] = st["mean"] / res["bf16_same_shape"]["ms_per_step"]["mean"]
+    del db
+    torch.cuda.empty_cache()
+    if cpu and not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = cpu_baseline(name, budget_s=4.0)
+    return res
 
 
-def run_long(args):
-    """The long workload as its decode loop: every step appends one token per
-    sequence with page reallocation and tag bumps; even steps validate with
-    0.01% of expected tags made stale (those requests abort for that step), odd
-    steps skip the check.  Step time = device time of append + validate +
-    decode replayed from a CUDA graph; bytes count decoded (non-aborted) rows."""
-    rank, world, local = dist_setup(args)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
+def assert_no_device_error():
     import fp8_kv_paged_kvq_b200 as kvq
-    from fp8_kv_paged_kvq_b200 import build as kvq_build
-    from fp8_kv_paged_kvq_b200 import workloads as W
-    from fp8_kv_paged_kvq_b200.pipeline import DecodeLoop
-    if rank == 0:
-        kvq_build.build()
-    barrier(world)
-    spec = W.spec_by_name("long")
-    wl = W.make_workload(spec, seed=0, device=dev)
-    steps = args.loop_steps
-    loop = DecodeLoop(wl, steps, device=dev, num_ctas=args.num_ctas)
-    loop.batch.prefill()
-    torch.cuda.synchronize()
-    row = spec.num_kv_heads * (spec.head_dim_k + spec.head_dim_v)
-    stream = torch.cuda.Stream(device=dev)
-    recs = []
-    with torch.cuda.stream(stream):
-        loop.capture(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        sampler = ClockSampler(local)
-        with sampler:
-            for ls in W.loop_steps(wl, steps):
-                # kind 0: check + stale tags, 1: clean check, 2: no check; the
-                # second half of each six-step cycle replays the graphs with
-                # events between the kernels, for the per-kernel breakdown
-                kind = ls.step % 3
-                detailed = (ls.step // 3) % 2 == 1
-                chk = kind != 2
-                idx = loop.prepare(ls, chk, inject_stale=(kind == 0))
-                ev = loop.run(chk, stream, detailed)
-                loop.restore(idx)
-                torch.cuda.synchronize()
-                ms_step = ev[0].elapsed_time(ev[-1])
-                parts = tuple(ev[i].elapsed_time(ev[i + 1]) for i in range(3)) if detailed else (0, 0, 0)
-                aborted = {b for b, _ in ls.stale} if kind == 0 else set()
-                kv = sum(int(ls.seq_lens[b]) for b in range(spec.B) if b not in aborted) * row
-                recs.append((kind, detailed, ms_step) + parts + (kv, len(aborted)))
     assert kvq.device_error() == 0, "device-side wait timed out"
-    kind = np.array([r[0] for r in recs])
-    det = np.array([r[1] for r in recs])
-    ms = np.array([r[2] for r in recs])
-    t_app = np.array([r[3] for r in recs])
-    t_val = np.array([r[4] for r in recs])
-    t_dec = np.array([r[5] for r in recs])
-    kv = np.array([r[6] for r in recs], dtype=np.float64)
-    # the tracker's view must match what the device did
-    host_tags = loop.tracker.tags
-    dev_tags = loop.batch.cache.page_tags.cpu().numpy().view(np.uint32)
-    tags_ok = bool(np.array_equal(host_tags, dev_tags))
-    def mean(x):
-        return float(max_over_ranks(float(np.mean(x)), world))
-    plain = ~det                                  # steps timed only at their boundaries
-    step_clean, step_nochk = mean(ms[plain & (kind == 1)]), mean(ms[plain & (kind == 2)])
-    # in the detailed graphs the no-check step records the same events around an
-    # empty slot: its gap is the event overhead, subtracted from the validate slot
-    val = mean(t_val[det & (kind == 1)]) - mean(t_val[det & (kind == 2)])
-    gbs = whole_job_gbs(world, kv[plain].sum(), max_over_ranks(float(ms[plain].sum()), world))
-    hbm, hbm_kind = peaks()
-    line = {
-        "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
-        "warmup": 1, "ms_per_step": float(ms[plain].mean()), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16 mma / f32 accumulate (e4m3 cache)", "data": "synthetic",
-        "config": {"workload": workload_desc("long"),
-                   "loop": f"{steps} steps: append 1 token/seq with page reallocation + tag "
-                           "bump; steps cycle validate+stale tags / validate / no validation",
-                   "l2": "inputs exceed L2: >3 GB of cache read per step",
-                   "timing": "CUDA graph per step between CUDA events; step time and value "
-                             "from the half of the steps with events only around the step"},
-        "decode_tokens_per_s": world * spec.B / (ms[plain].mean() * 1e-3),
-        "hbm_frac_of_step": gbs / world / hbm,
-        "ms_per_step_with_validation": step_clean,
-        "ms_per_step_without_validation": step_nochk,
-        "ms_per_step_with_validation_and_stale_tags": mean(ms[plain & (kind == 0)]),
-        "p95_ms_with_validation": float(np.percentile(ms[plain & (kind == 1)], 95)),
-        "p95_ms_without_validation": float(np.percentile(ms[plain & (kind == 2)], 95)),
-        "ms_validate_kernel": val,
-        "ms_decode_with_validation": mean(t_dec[det & (kind == 1)]),
-        "ms_decode_without_validation": mean(t_dec[det & (kind == 2)]),
-        "ms_decode_with_stale_aborts": mean(t_dec[det & (kind == 0)]),
-        "ms_append": mean(t_app[det]),
-        "validate_overhead_pct": 100.0 * (step_clean - step_nochk) / step_nochk,
-        "validate_overhead_note": "steps cycle: validate with 0.01% stale tags / validate with "
-                                  "clean tags / no validation; overhead compares the last two, "
-                                  "each timed only at the step's boundaries",
-        "aborted_requests_per_stale_step": float(np.mean([r[7] for r in recs if r[0] == 0])),
-        "pages_reallocated": int(sum(len(l.new_pages) for l in W.loop_steps(wl, steps))),
-        "host_tracker_matches_device_tags": tags_ok,
-        "clocks": sampler.summary(), "gpu_launches": int(4 * np.sum(kind != 2) + 3 * np.sum(kind == 2)),
-    }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
 
 
 def run_e2e(db, args, stream, kv_bytes, world):
     """Same step through the public API, its inputs copied from pinned host
     memory and its results (out, lse, abort mask) read back, every step:
-    - value: two CUDA graphs (DecodeBatch.capture_io_pipelined) replayed in
-      turn; each replay runs one step while copying in the next step's inputs
-      and copying out the previous step's results on side streams;
-    - serial: one graph per step holding its copies, append, validate, decode
-      and read-back in order (DecodeBatch.capture_io_step);
-    - eager: the same calls issued one by one from Python each step."""
-    K = args.e2e_steps
+    two CUDA graphs (DecodeBatch.capture_io_pipelined) replayed in turn; each
+    replay runs one step while copying in the next step's inputs and copying
+    out the previous step's results on side streams."""
     names = [n for n in db.IO_IN if getattr(db, n) is not None]
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype).pin_memory()
     host_in = [{n: getattr(db, n).detach().cpu().pin_memory() for n in names} for _ in range(2)]
     host_out = [{n: pin(getattr(db, n)) for n in db.IO_OUT} for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host_in[0].values())
     d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
-
-    def one():
-        for n, h in host_in[0].items():
-            getattr(db, n).copy_(h, non_blocking=True)
-        db.step(check_tags=True, stream=stream)
-        for n, h in host_out[0].items():
-            h.copy_(getattr(db, n), non_blocking=True)
-
-    def timed(fns):
-        for i in range(6):
-            fns[i % len(fns)]()
-        barrier(world)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(K):
-            fns[i % len(fns)]()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        return max_over_ranks(e0.elapsed_time(e1) / K, world)
-
     with torch.cuda.stream(stream):
-        ms_eager = timed([one])
-        g = db.capture_io_step(host_in[0], host_out[0], stream)
-        ms_serial = timed([g.replay])
-        del g
         ga, gb = db.capture_io_pipelined(host_in, host_out, stream)
-        ms = timed([ga.replay, gb.replay])
+        flip = [0]
+
+        def one():
+            (ga if flip[0] == 0 else gb).replay()
+            flip[0] ^= 1
+        for _ in range(6):
+            one()
+        barrier(world)
+        t = time_replays(one, stream, args.min_seconds / 2)
         del ga, gb
-    gbs = lambda m: whole_job_gbs(world, kv_bytes, m)
-    return {"value": gbs(ms), "unit": "GB/s",
+    ms = max_over_ranks(float(t.mean()), world)
+    return {"value": whole_job_gbs(world, kv_bytes, ms), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "steps": K, "path": "python binding -> C ABI; two CUDA graphs in turn, each a step "
-                                "(append, validate, decode) with the next step's host->device "
-                                "copies and the previous step's device->host copies beside it",
-            "serial": {"value": gbs(ms_serial), "ms_per_step": ms_serial,
-                       "path": "one CUDA graph per step: copies in, step, copies out, in order"},
-            "eager": {"value": gbs(ms_eager), "ms_per_step": ms_eager,
-                      "path": "the same calls launched one by one from Python"}}
+            "steps": int(t.size),
+            "path": "python binding -> C ABI; two CUDA graphs in turn, each a step (append, "
+                    "validate, decode) with the next step's host->device copies and the "
+                    "previous step's device->host copies beside it"}
 
 
 def run_bf16(wl_fp8, args, stream, world, dev):
@@ -669,7 +562,7 @@ def run_bf16(wl_fp8, args, stream, world, dev):
     db = DecodeBatch(wl_fp8, device=dev, num_ctas=args.num_ctas, kv_dtype=W.BF16)
     db.prefill()
     with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
+        for _ in range(3):
             db.step(check_tags=True, stream=stream)
         g = capture(lambda: db.step(check_tags=True, stream=stream), stream)
         gd = capture(lambda: db.decode(use_abort=True, stream=stream), stream)
@@ -677,20 +570,25 @@ def run_bf16(wl_fp8, args, stream, world, dev):
             g.replay()
             gd.replay()
         barrier(world)
-        ms = max_over_ranks(time_graph(g, args.steps, stream), world)
-        msd = max_over_ranks(time_graph(gd, args.steps, stream), world)
+        t = stats(time_replays(g.replay, stream, args.min_seconds))
+        td = stats(time_replays(gd.replay, stream, args.min_seconds))
+    ms = max_over_ranks(t["mean"], world)
+    msd = max_over_ranks(td["mean"], world)
     kv = 2 * wl_fp8.kv_bytes_read()
     hbm, _ = peaks()
-    res = {"ms_per_step": ms, "kv_gbs": whole_job_gbs(world, kv, ms),
-           "decode_ms_per_launch": msd, "decode_kv_gbs": kv / (msd * 1e-3) / 1e9,
+    spec16 = W.Spec(**{**wl_fp8.spec.__dict__, "kv_dtype": W.BF16})
+    lens = np.minimum(wl_fp8.seq_lens, wl_fp8.max_pages * spec16.page_size)
+    res = {"ms_per_step": t, "kv_gbs": whole_job_gbs(world, kv, ms),
+           "ms_decode_call": td, "decode_kv_gbs": kv / (msd * 1e-3) / 1e9,
            "decode_frac_of_hbm": kv / (msd * 1e-3) / 1e9 / hbm,
+           "roofline": decode_roofline(spec16, lens, msd, None),
            "decode_tokens_per_s": world * wl_fp8.B / (ms * 1e-3)}
     del g, gd, db
     torch.cuda.empty_cache()
     return res
 
 
-def run_bulk_append(spec, dev, stream, tokens=65536, iters=20):
+def run_bulk_append(spec, dev, stream, tokens=65536):
     """Bulk quantize: a prompt's worth of BF16 K/V (tokens x Hkv x D) through
     kvq_append into FP8 pages scattered by a random page permutation, as at
     the prefill -> decode hand-over.  Algorithmic bytes: the BF16 reads, the
@@ -707,8 +605,6 @@ def run_bulk_append(spec, dev, stream, tokens=65536, iters=20):
     # powers of two, so every value takes the checked product quotient
     kvq.scale_from_amax(kvq.amax(k, True), out=cache.k_scale)
     kvq.scale_from_amax(kvq.amax(v, True), out=cache.v_scale)
-    pow2 = bool(((cache.k_scale.view(torch.int32) & 0x7FFFFF) == 0).any() or
-                ((cache.v_scale.view(torch.int32) & 0x7FFFFF) == 0).any())
     perm = torch.randperm(pages, device=dev, generator=g).to(torch.int32)
     t = torch.arange(tokens, device=dev, dtype=torch.int32)
     slots = (perm[t // ps] * ps + t % ps).contiguous()
@@ -716,14 +612,223 @@ def run_bulk_append(spec, dev, stream, tokens=65536, iters=20):
         for _ in range(3):
             kvq.append(cache, k, v, slots, stream=stream)
         gr = capture(lambda: kvq.append(cache, k, v, slots, stream=stream), stream)
-        ms = time_graph(gr, iters, stream)
+        t = stats(time_replays(gr.replay, stream, 0.2))
     nbytes = tokens * H * (Dk + Dv) * 3 + tokens * 4
     hbm, kind = peaks()
     del gr
-    return {"tokens": tokens, "ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
-            "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm, "peak_kind": kind,
+    return {"tokens": tokens, "ms": t, "gbs": nbytes / (t["mean"] * 1e-3) / 1e9,
+            "frac_of_hbm": nbytes / (t["mean"] * 1e-3) / 1e9 / hbm, "peak_kind": kind,
             "bytes": nbytes, "note": "bf16 K/V read + e4m3 codes written + slot mapping",
-            "scales": "per head, amax / 448 of the data" + (" (some powers of two)" if pow2 else "")}
+            "scales": "per head, amax / 448 of the data"}
+
+
+# ---------------------------------------------------------------------------
+# the long workload: the 1,000-step loop
+# ---------------------------------------------------------------------------
+def run_long(args, rank, world, local, dev):
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    from fp8_kv_paged_kvq_b200.pipeline import CLEAN, NOCHECK, STALE, DecodeLoop
+    spec = W.spec_by_name("long")
+    wl = W.make_workload(spec, seed=0, device=dev)
+    n = args.loop_steps
+    loop = DecodeLoop(wl, n, device=dev, num_ctas=args.num_ctas)
+    loop.batch.prefill()
+    torch.cuda.synchronize()
+    loop.snapshot_tags()
+    stream = torch.cuda.Stream(device=dev)
+    # kinds cycle stale / clean / no check; every other cycle of three steps
+    # runs each call as its own graph with events between them (the decode
+    # call's time), the others as one graph per step with events only at the
+    # step's boundaries (the step times)
+    kinds = [(STALE, CLEAN, NOCHECK)[i % 3] for i in range(n)]
+    detailed = [(i // 3) % 2 == 1 for i in range(n)]
+    loop.capture(stream, kinds, detailed)
+    row = spec.num_kv_heads * (spec.head_dim_k + spec.head_dim_v)
+    lens = np.stack([ls.seq_lens for ls in loop.plan]).astype(np.int64)
+    aborted = [{b for b, _ in ls.stale} if kinds[ls.step] == STALE else set() for ls in loop.plan]
+    kv = np.array([sum(int(lens[i, b]) for b in range(spec.B) if b not in aborted[i]) * row
+                   for i in range(n)], np.float64)
+    alg_dec = np.array([decode_alg_bytes(spec, [lens[i, b] for b in range(spec.B)
+                                                if b not in aborted[i]]) for i in range(n)])
+
+    def new_events():
+        return [[torch.cuda.Event(enable_timing=True) for _ in range(4 if d else 2)]
+                for d in detailed]
+
+    evsets = [new_events(), new_events()]
+    rec = []
+
+    def harvest(evs):
+        for i, ev in enumerate(evs):
+            t = [ev[j].elapsed_time(ev[j + 1]) for j in range(len(ev) - 1)]
+            rec.append((i, sum(t)) + tuple(t if len(t) == 3 else (0.0, 0.0, 0.0)))
+
+    for _ in range(max(3, args.warmup)):
+        loop.replay_pass(stream)
+    torch.cuda.synchronize()
+    loop.batch.cache.page_tags.copy_(loop.tags0)
+    barrier(world)
+    sampler = ClockSampler(local)
+    t_wall = time.perf_counter()
+    with sampler:
+        # passes alternate between two event sets: pass p + 1 is queued before
+        # pass p's events are read, so the device never waits for the host
+        for p in range(args.steps):
+            loop.replay_pass(stream, evsets[p % 2])
+            if p > 0:
+                evsets[(p - 1) % 2][-1][-1].synchronize()
+                harvest(evsets[(p - 1) % 2])
+        torch.cuda.synchronize()
+        harvest(evsets[(args.steps - 1) % 2])
+    barrier(world)
+    wall = time.perf_counter() - t_wall
+    assert_no_device_error()
+    tags_ok = bool(np.array_equal(loop.batch.cache.page_tags.cpu().numpy().view(np.uint32),
+                                  loop.final_tags()))
+    idx = np.array([r[0] for r in rec])
+    ms = np.array([r[1] for r in rec])
+    t_app, t_val, t_dec = (np.array([r[k] for r in rec]) for k in (2, 3, 4))
+    kind = np.array([kinds[i] for i in idx])
+    det = np.array([detailed[i] for i in idx])
+    plain = ~det
+    clean, nochk, stale = plain & (kind == CLEAN), plain & (kind == NOCHECK), plain & (kind == STALE)
+    dclean = det & (kind == CLEAN)
+    m = lambda x: max_over_ranks(float(x), world)
+    ms_clean = m(ms[clean].mean())
+    value = whole_job_gbs(world, kv[idx[clean]].sum(), m(ms[clean].sum()))
+    sc, sn, ss = stats(ms[clean]), stats(ms[nochk]), stats(ms[stale])
+    # decode call (decode kernel + combine) timed between events in the clean
+    # detailed steps: algorithmic bytes / time, summed over those steps
+    dec_ms = m(t_dec[dclean].sum()) / dclean.sum()
+    dec_bytes = alg_dec[idx[dclean]].mean()
+    roof = decode_roofline(spec, lens[n // 2], dec_ms, measured_traffic("long", 0),
+                           alg_bytes=dec_bytes)
+    roof["note"] = ("decode call between events inside the clean steps of the timed passes; "
+                    "algorithmic bytes and time averaged over those steps")
+    hbm, _ = peaks()
+    launches = sum(3 if k == NOCHECK else 4 for k in kinds) * args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": ms_clean, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
+        "config": {"workload": workload_desc("long"),
+                   "loop": f"{n} decode steps per pass: append 1 token/seq with page "
+                           "reallocation + tag bump, then the tag check, then decode; steps "
+                           "cycle check with 0.01% stale tags / clean check / no check",
+                   "steps_and_warmup": f"passes over the {n}-step loop (each pass resets the "
+                                       "live tags and repeats the same tag history)",
+                   "ms_per_step": "one decode step (append + validate + decode), mean over "
+                                  "the clean steps",
+                   "value": "KV bytes of the clean steps / their device time",
+                   "l2": "inputs exceed L2: >3 GB of cache read per step",
+                   "timing": "one CUDA graph per step, CUDA events at step boundaries, "
+                             "max over ranks",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "decode_tokens_per_s": world * spec.B / (ms_clean * 1e-3),
+        "hbm_frac_of_step": value / world / hbm,
+        "ms_per_step_stats": sc,
+        "ms_per_step_without_validation": sn,
+        "ms_per_step_with_stale_tags": ss,
+        "validate_overhead_pct": 100.0 * (sc["mean"] - sn["mean"]) / sn["mean"],
+        "validate_overhead_p95_pct": 100.0 * (sc["p95"] - sn["p95"]) / sn["p95"],
+        "validate_overhead_median_pct": 100.0 * (sc["median"] - sn["median"]) / sn["median"],
+        "validate_overhead_note": "clean steps (check on, every tag right) against steps "
+                                  "without the check, each timed at its boundaries only",
+        "ms_decode_call": stats(t_dec[dclean]),
+        "ms_validate_call": stats(t_val[dclean]),
+        "ms_append_call": stats(t_app[dclean]),
+        "aborted_requests_per_stale_step": float(np.mean([len(a) for a in aborted if a]
+                                                         or [0])),
+        "pages_reallocated_per_pass": int(sum(len(ls.new_pages) for ls in loop.plan)),
+        "host_tracker_matches_device_tags": tags_ok,
+        "roofline": roof,
+        "gpu_launches": launches,
+        "timed_region_s": wall,
+        "clocks": sampler.summary(),
+    }
+    if not args.no_e2e:
+        line["e2e"] = run_long_e2e(loop, stream, world, row, spec)
+    del loop
+    torch.cuda.empty_cache()
+    return line
+
+
+def run_long_e2e(loop, stream, world, row, spec):
+    """The loop through the public API with host buffers: every step's inputs
+    (query, new K/V, slots, lengths, reallocated pages, new block-table and
+    expected-tag entries) copied from pinned host memory and its results
+    (out, lse, abort mask, abort count) read back, host traffic overlapped
+    with the neighbouring steps.  Every step runs the clean check."""
+    io = loop.io_setup(stream)
+    loop.io_pass(stream, steps=50)                    # warm-up
+    barrier(world)
+    e0, e1, counts = loop.io_pass(stream)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world)
+    lens = np.stack([ls.seq_lens for ls in loop.plan]).astype(np.int64)
+    kv = float(lens.sum()) * row
+    n = len(counts)
+    assert all(c == 0 for c in counts), "clean steps must abort nothing"
+    return {"value": whole_job_gbs(world, kv, ms_total), "unit": "GB/s",
+            "h2d_bytes_per_step": io["h2d_bytes_per_step"],
+            "d2h_bytes_per_step": io["d2h_bytes_per_step"],
+            "ms_per_step": ms_total / n, "steps": n,
+            "path": "python binding -> C ABI; two CUDA graphs in turn, each a step (block-table "
+                    "entries, append, validate, decode) with the next step's host->device "
+                    "copies and the previous step's device->host copies beside it; every "
+                    "step's abort count read back and checked"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    rank, world, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import fp8_kv_paged_kvq_b200 as kvq
+    from fp8_kv_paged_kvq_b200 import build as kvq_build
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    if rank == 0:
+        kvq_build.build()
+    barrier(world)
+    kvq.lib()
+    stream = torch.cuda.Stream(device=dev)
+    if args.workload == "long":
+        line = run_long(args, rank, world, local, dev)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline("long", budget_s=8.0)
+        extra = [] if args.no_extra else ["gqa", "ragged", "wide"]
+    else:
+        # a single decode batch as the headline: K timed steps after W warm-up steps
+        res = measure_batch(args.workload, args, dev, stream, world, e2e=not args.no_e2e,
+                            cpu=False)
+        st = res["ms_per_step"]
+        line = {"metric": METRIC, "value": res["kv_gbs"], "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": st["mean"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": DTYPE, "data": "synthetic",
+                "config": {"workload": res["workload"],
+                           "step": "kvq_append + kvq_validate + kvq_decode",
+                           "timing": res["timing"],
+                           "parallelism": "replicas" if world > 1 else "single GPU"}}
+        line.update({k: v for k, v in res.items() if k not in ("workload", "kv_gbs")})
+        line["gpu_launches"] = (2 + (3 if is_wide(W.spec_by_name(args.workload)) else 2)) * st["n"]
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=8.0)
+        extra = []
+    if extra:
+        line["configs"] = {}
+        for name in extra:
+            line["configs"][name] = measure_batch(name, args, dev, stream, world,
+                                                  e2e=(name == "gqa"), bf16=(name != "wide"))
+        s = W.spec_by_name("gqa")
+        line["bulk_append"] = run_bulk_append(s, dev, stream)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
 
 
 def run_sweep(args):
@@ -733,7 +838,6 @@ def run_sweep(args):
     format (cache bytes per token read from the allocated pages)."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    import fp8_kv_paged_kvq_b200 as kvq
     from fp8_kv_paged_kvq_b200 import build as kvq_build
     from fp8_kv_paged_kvq_b200 import workloads as W
     from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch
@@ -760,14 +864,14 @@ def run_sweep(args):
                 for _ in range(3):
                     db.decode(use_abort=False, stream=stream)
                 gd = capture(lambda: db.decode(use_abort=False, stream=stream), stream)
-                ms = time_graph(gd, args.steps, stream)
+                t = stats(time_replays(gd.replay, stream, args.min_seconds))
             kv = wl.kv_bytes_read()               # bytes of this cache format
-            row[dt] = {"ms": ms, "kv_gbs": kv / (ms * 1e-3) / 1e9,
-                       "frac_of_hbm": kv / (ms * 1e-3) / 1e9 / hbm,
-                       "decode_tokens_per_s": B / (ms * 1e-3)}
+            row[dt] = {"ms": t, "kv_gbs": kv / (t["mean"] * 1e-3) / 1e9,
+                       "frac_of_hbm": kv / (t["mean"] * 1e-3) / 1e9 / hbm,
+                       "decode_tokens_per_s": B / (t["mean"] * 1e-3)}
             del gd, db
             torch.cuda.empty_cache()
-        row["fp8_over_bf16_time"] = row[W.FP8]["ms"] / row[W.BF16]["ms"]
+        row["fp8_over_bf16_time"] = row[W.FP8]["ms"]["mean"] / row[W.BF16]["ms"]["mean"]
         rows.append(row)
     line = {"sweep": "gqa shape, 8,192 tokens per sequence, decode call only",
             "rows": rows,
@@ -775,8 +879,7 @@ def run_sweep(args):
                          "fp8_bytes_per_token": per_token[W.FP8],
                          "bf16_bytes_per_token": per_token[W.BF16],
                          "fp8_tokens": int(budget // per_token[W.FP8]),
-                         "bf16_tokens": int(budget // per_token[W.BF16])},
-            "steps": args.steps}
+                         "bf16_tokens": int(budget // per_token[W.BF16])}}
     print(json.dumps(line), flush=True)
 
 
@@ -786,8 +889,6 @@ def main():
         run_reference(args)
     elif args.sweep:
         run_sweep(args)
-    elif args.workload == "long":
-        run_long(args)
     else:
         run_ours(args)
 

@@ -6,7 +6,7 @@ oracle's own quantization, abort masks bit-exact, and sampled output rows
 The long workload runs its whole 1,000-step loop: every step's abort mask is
 compared with the oracle's, whose expected tags come from the oracle's own
 tag state (a page's tag right after the oracle's append reallocated it), not
-from the library's host tracker.
+from the library's host tracker; every output row is compared at three steps.
 """
 import numpy as np
 import pytest
@@ -15,7 +15,7 @@ import torch
 import oracle
 import fp8_kv_paged_kvq_b200 as kvq
 from fp8_kv_paged_kvq_b200 import workloads as W
-from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch, DecodeLoop
+from fp8_kv_paged_kvq_b200.pipeline import NOCHECK, STALE, DecodeBatch, DecodeLoop
 from tests import oracle_side as OS
 from tests.test_gpu_parity import assert_decode_close
 
@@ -77,7 +77,38 @@ def test_full_size_step(name, kv):
     assert kvq.device_error() == 0
 
 
+def test_wide_whole_sequences_all_heads():
+    """The wide batch in the launch configuration bench.py times: every query
+    head of four whole sequences, the first and last of the batch among them,
+    so that the first and last pieces of the split are covered."""
+    spec = W.spec_by_name("wide")
+    wl = W.make_workload(spec, seed=0, device="cuda")
+    db = DecodeBatch(wl)
+    db.prefill()
+    out, lse = db.step(check_tags=True)
+    torch.cuda.synchronize()
+    oc = OS.new_cache(wl)
+    OS.fill(wl, oc)
+    mask = oracle.validate(oc.page_tags, wl.block_table, wl.expected_tags, wl.seq_lens,
+                           spec.page_size)
+    assert np.array_equal(db.abort.cpu().numpy(), mask)
+    seqs = (0, 1, 31, spec.B - 1)
+    rows = np.array([b * spec.num_q_heads + h for b in seqs for h in range(spec.num_q_heads)],
+                    np.int32)
+    ro, rl = OS.decode(wl, oc, abort=mask, rows=rows)
+    ri = torch.from_numpy(rows).long().cuda()
+    assert_decode_close(out.reshape(-1, spec.head_dim_v)[ri], lse.reshape(-1)[ri], ro, rl,
+                        "wide whole sequences")
+    assert kvq.device_error() == 0
+
+
 def test_long_loop_1000_steps():
+    """The 1,000-step loop as bench.py runs it (one CUDA graph per step over
+    inputs laid out on the device).  Even steps check the tags with stale
+    entries injected, odd steps skip the check.  Every step's abort mask is
+    compared with the oracle's; every output row (all 64 sequences x 64
+    query heads) is compared at steps 0, 1 and 999; the final tags, block
+    tables and codes of the whole cache are compared at the end."""
     spec = W.spec_by_name("long")
     steps = 1000
     wl = W.make_workload(spec, seed=0, device="cuda")
@@ -85,6 +116,11 @@ def test_long_loop_1000_steps():
     loop.batch.cache.k_pages.fill_(0xCD)      # same canary as the oracle's cache
     loop.batch.cache.v_pages.fill_(0xCD)
     loop.batch.prefill()
+    torch.cuda.synchronize()
+    loop.snapshot_tags()
+    kinds = [STALE if i % 2 == 0 else NOCHECK for i in range(steps)]
+    stream = torch.cuda.Stream()
+    loop.capture(stream, kinds)
     # oracle side: its own cache, block table and expected tags
     oc = OS.new_cache(wl)
     hist = [(OS.bf16_bits(k), OS.bf16_bits(v), sl) for k, v, sl in wl.hist_chunks()]
@@ -99,48 +135,40 @@ def test_long_loop_1000_steps():
     oexp = np.zeros((spec.B, cap), np.uint32)
     oexp[:, : wl.max_pages] = np.where(wl.block_table >= 0,
                                        oc.page_tags[np.maximum(wl.block_table, 0)], 0)
-    check_rows = {0, 1, steps - 1}
-    rows = np.array([b * spec.num_q_heads + h for b in (0, 1, 2, 3, 10, 63) for h in (0, 37)],
-                    np.int32)
-    stream = torch.cuda.Stream()
+    check_steps = {0, 1, steps - 1}
+    q = OS.bf16_bits(wl.q())
     n_aborts = 0
-    with torch.cuda.stream(stream):
-        loop.capture(stream)
-        for ls in W.loop_steps(wl, steps):
-            chk = ls.step % 2 == 0
-            idx = loop.prepare(ls, chk)
-            loop.run(chk, stream)
-            loop.restore(idx)
-            torch.cuda.synchronize()
-            # oracle step
-            k, v = W.loop_tokens(wl, ls.step)
-            pages = [p for _, _, p in ls.new_pages]
-            oracle.append(oc, OS.bf16_bits(k), OS.bf16_bits(v), ls.slots,
-                          realloc_pages=np.array(pages, np.int32) if pages else None)
-            for b, i, p in ls.new_pages:
-                obt[b, i] = p
-                oexp[b, i] = oc.page_tags[p]
-            if chk:
-                e = oexp.copy()
-                for b, i in ls.stale:
-                    e[b, i] ^= np.uint32(1)
-                m = oracle.validate(oc.page_tags, obt, e, ls.seq_lens, spec.page_size)
-                got = loop.batch.abort.cpu().numpy()
-                assert np.array_equal(got, m), ls.step
-                assert set(np.nonzero(m)[0].tolist()) == {b for b, _ in ls.stale}
-                n_aborts += int(m.sum())
-            else:
-                m = None
-            if ls.step in check_rows:
-                q = OS.bf16_bits(wl.q())
-                ro, rl = oracle.decode(oc, q, obt, ls.seq_lens, m, wl.sm_scale, rows=rows)
-                ri = torch.from_numpy(rows).long().cuda()
-                o = loop.batch.out.reshape(-1, spec.head_dim_v)[ri]
-                l = loop.batch.lse.reshape(-1)[ri]
-                assert_decode_close(o, l, ro, rl, f"step {ls.step}")
+    for ls in W.loop_steps(wl, steps):
+        chk = kinds[ls.step] == STALE
+        loop.replay_step(ls.step, stream)
+        torch.cuda.synchronize()
+        # oracle step
+        k, v = W.loop_tokens(wl, ls.step)
+        pages = [p for _, _, p in ls.new_pages]
+        oracle.append(oc, OS.bf16_bits(k), OS.bf16_bits(v), ls.slots,
+                      realloc_pages=np.array(pages, np.int32) if pages else None)
+        for b, i, p in ls.new_pages:
+            obt[b, i] = p
+            oexp[b, i] = oc.page_tags[p]
+        m = None
+        if chk:
+            e = oexp.copy()
+            for b, i in ls.stale:
+                e[b, i] ^= np.uint32(1)
+            m = oracle.validate(oc.page_tags, obt, e, ls.seq_lens, spec.page_size)
+            got = loop.batch.abort.cpu().numpy()
+            assert np.array_equal(got, m), ls.step
+            assert set(np.nonzero(m)[0].tolist()) == {b for b, _ in ls.stale}
+            n_aborts += int(m.sum())
+        if ls.step in check_steps:
+            ro, rl = oracle.decode(oc, q, obt, ls.seq_lens, m, wl.sm_scale)
+            assert_decode_close(loop.batch.out.reshape(-1, spec.head_dim_v),
+                                loop.batch.lse.reshape(-1), ro, rl, f"step {ls.step}")
     assert n_aborts > 0
     assert np.array_equal(loop.batch.cache.page_tags.cpu().numpy().view(np.uint32), oc.page_tags)
-    assert np.array_equal(loop.tracker.tags, oc.page_tags)
+    assert np.array_equal(loop.final_tags(), oc.page_tags)
+    assert np.array_equal(loop.tracker.block_table, obt)
+    assert np.array_equal(loop.tracker.expected, oexp)
     assert np.array_equal(loop.batch.cache.k_pages.cpu().numpy(), oc.k_pages)
     assert np.array_equal(loop.batch.cache.v_pages.cpu().numpy(), oc.v_pages)
     assert kvq.device_error() == 0
