@@ -8,10 +8,28 @@
 // Modellbereitstellung senkt Speicherbedarf, doch Sicherheit wird zum
 // Prüfstein" (remio.ai), section "Sicherheit gemeinsamer KV-Caches wird zum
 // Produktionsthema").
+#include <mutex>
+
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
+
+template <typename K>
+cudaError_t prefer_max_shared(K* kernel) {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
 
 // ---------------------------------------------------------------------------
 // amax: one block per (row chunk, head or all heads); 16-byte loads.
@@ -421,6 +439,8 @@ cudaError_t launch_append(const CacheView& c, const uint16_t* k_new, const uint1
   a.token_blocks = static_cast<int32_t>((warps + kAppendWarps - 1) / kAppendWarps);
   const int32_t blocks = a.token_blocks + (n_realloc > 0 ? 1 : 0);
   if (blocks == 0) return cudaSuccess;
+  const cudaError_t e = prefer_max_shared(append_kernel);
+  if (e != cudaSuccess) return e;
   append_kernel<<<blocks, kAppendWarps * 32, 0, stream>>>(a);
   return cudaGetLastError();
 }

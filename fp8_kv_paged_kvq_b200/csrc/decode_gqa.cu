@@ -627,11 +627,12 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
 // The decode launch gave its units to N = min(num_ctas, U) CTAs, CTA c taking
 // [c*U/N, (c+1)*U/N), so unit u belongs to CTA ((u+1)*N - 1) / U and the
 // pieces of a segment with units [S, E) are exactly the CTAs cs..ce that own
-// S and E - 1, every one of them non-empty.  Warp w turns the partial lse
-// values of its heads into a maximum M and a sum L over any number of
-// pieces; the block then forms out = sum_k exp(lse_k - M) / L * o_k with
-// coalesced 16-byte loads, taking the pieces in chunks of kCombChunk whose
-// weights it stages in shared memory.
+// S and E - 1, every one of them non-empty.  With up to kCombFast pieces
+// each thread loads its outputs' partials from every piece in one round and
+// merges them itself: out = sum_k exp(lse_k - M) / L * o_k with M the
+// largest lse_k and L the sum of exp(lse_k - M).  With more pieces, warp w
+// first forms M and L for its heads, and the block then takes the pieces in
+// chunks of kCombChunk whose weights it stages in shared memory.
 // ---------------------------------------------------------------------------
 struct CombineParams {
   const int32_t* ws_pre;
@@ -647,6 +648,7 @@ constexpr int kCombHeads = 32;        // heads per block at most
 constexpr int kCombChunk = 64;        // pieces whose weights are staged at once
 constexpr int kCombOutputs = 4096;    // outputs per block (heads_per_block * Dv) at most
 constexpr int kCombPerThread = kCombOutputs / 4 / kCombThreads;   // float4 outputs per thread
+constexpr int kCombFast = 4;          // pieces merged from registers in one round of loads
 
 // CTA of a launch with N working CTAs over U units that owns unit u.
 __device__ __forceinline__ int64_t owner_cta(int64_t u, int64_t N, int64_t U) {
@@ -676,6 +678,73 @@ __global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const Combine
   const int64_t cs = owner_cta(S, N, U);
   const int np = static_cast<int>(owner_cta(E - 1, N, U) - cs + 1);
   const int64_t slot0 = cs + seg;               // slot of piece k: slot0 + k
+  const int dq = p.Dv >> 2;                     // outputs in groups of four dims
+  const int n4 = nh * dq;
+  const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+  if (np <= kCombFast) {
+    // Few pieces: thread t loads, in one round, the partial outputs of its
+    // groups t, t + kCombThreads, ... and the partial lse of their heads
+    // from every piece, and merges them on its own.
+    float4 o[kCombPerThread][kCombFast];
+    float a[kCombPerThread][kCombFast];
+#pragma unroll
+    for (int r = 0; r < kCombPerThread; ++r) {
+      const int i4 = threadIdx.x + r * kCombThreads;
+      const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
+#pragma unroll
+      for (int k = 0; k < kCombFast; ++k) {
+        if (i4 < n4 && k < np) {
+          const int64_t row = (slot0 + k) * p.G + h0 + hh;
+          o[r][k] = *reinterpret_cast<const float4*>(p.ws_o + row * p.Dv + d);
+          a[r][k] = p.ws_lse[row];
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kCombPerThread; ++r) {
+      const int i4 = threadIdx.x + r * kCombThreads;
+      if (i4 >= n4) continue;
+      const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
+      float4 acc = o[r][0];                      // a single piece is copied bit for bit
+      float lse_h = a[r][0];
+      if (np > 1) {
+        float M = a[r][0];
+#pragma unroll
+        for (int k = 1; k < kCombFast; ++k)
+          if (k < np) M = fmaxf(M, a[r][k]);
+        float L = 0.0f, w[kCombFast];
+#pragma unroll
+        for (int k = 0; k < kCombFast; ++k) {
+          w[k] = k < np ? __expf(a[r][k] - M) : 0.0f;
+          L += w[k];
+        }
+        const float inv = 1.0f / L;
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < kCombFast; ++k) {
+          if (k < np) {
+            const float wk = w[k] * inv;
+            acc.x += wk * o[r][k].x;
+            acc.y += wk * o[r][k].y;
+            acc.z += wk * o[r][k].z;
+            acc.w += wk * o[r][k].w;
+          }
+        }
+        lse_h = M + __logf(L);
+      }
+      if (lse && d == 0) lse[hh] = lse_h;
+      float* dst = out + hh * p.Dv + d;
+      if (vec_out) {
+        *reinterpret_cast<float4*>(dst) = acc;
+      } else {
+        dst[0] = acc.x;
+        dst[1] = acc.y;
+        dst[2] = acc.z;
+        dst[3] = acc.w;
+      }
+    }
+    return;
+  }
   __shared__ float m_sh[kCombHeads], inv_sh[kCombHeads];
   __shared__ float wts[kCombHeads][kCombChunk];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -694,27 +763,15 @@ __global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const Combine
     if (lane == 0) {
       m_sh[hh] = M;
       inv_sh[hh] = 1.0f / L;
-      if (lse) lse[hh] = np == 1 ? l[0] : M + __logf(L);
+      if (lse) lse[hh] = M + __logf(L);
     }
   }
-  // outputs in groups of four consecutive dims (Dv is a multiple of 4); thread
-  // t holds groups t, t + kCombThreads, ...
-  const int dq = p.Dv >> 2;
-  const int n4 = nh * dq;
+  // many pieces: thread t holds groups t, t + kCombThreads, ... and the
+  // pieces come in chunks whose weights are staged in shared memory
   float4 acc[kCombPerThread];
 #pragma unroll
   for (int r = 0; r < kCombPerThread; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (np == 1) {
-    // a single piece is copied bit for bit
-#pragma unroll
-    for (int r = 0; r < kCombPerThread; ++r) {
-      const int i4 = threadIdx.x + r * kCombThreads;
-      if (i4 < n4) {
-        const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
-        acc[r] = *reinterpret_cast<const float4*>(p.ws_o + (slot0 * p.G + h0 + hh) * p.Dv + d);
-      }
-    }
-  } else {
+  {
     __syncthreads();                             // m_sh, inv_sh
     for (int base = 0; base < np; base += kCombChunk) {
       const int nk = min(kCombChunk, np - base);
@@ -745,7 +802,6 @@ __global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const Combine
       __syncthreads();                           // wts reused by the next chunk
     }
   }
-  const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
 #pragma unroll
   for (int r = 0; r < kCombPerThread; ++r) {
     const int i4 = threadIdx.x + r * kCombThreads;

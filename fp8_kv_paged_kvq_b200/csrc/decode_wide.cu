@@ -877,6 +877,8 @@ cudaError_t launch_wide_decode(const DecodeArgs& a, const CUtensorMap& kqk,
   p.ws_lse = reinterpret_cast<float*>(ws + wl.off_lse);
   p.ws_o = reinterpret_cast<float*>(ws + wl.off_o);
   p.ws_q = ws + wl.off_extra;
+  e = prefer_max_shared(wide::wide_prep_kernel);
+  if (e != cudaSuccess) return e;
   e = launch_pdl(wide::wide_prep_kernel, dim3(2 * a.B + 1), dim3(wide::kPrepThreads), 0,
                  a.stream, p);
   if (e != cudaSuccess) return e;

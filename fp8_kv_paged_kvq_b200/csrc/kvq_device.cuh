@@ -429,12 +429,6 @@ __device__ __forceinline__ void st_shared_keep(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// Bring the line holding p into L2 (no register result; L2 is where global
-// memory is coherent, so a later load still sees every write made meanwhile).
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
-}
-
 // 16 bytes from the shared memory of a CTA of the cluster (address from mapa).
 // No memory clobber: volatile asm keeps its order against the barrier waits
 // (also volatile asm), while the compiler may still let several of these

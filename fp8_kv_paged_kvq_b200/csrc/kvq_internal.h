@@ -35,4 +35,13 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
                             int32_t* n_aborted, int32_t* first_bad, cudaStream_t stream);
 cudaError_t read_and_clear_error_flags(uint32_t* flags);
 
+// Ask for the largest shared-memory carveout for `kernel` on the current
+// device (once per device).  The small kernels launched just before a decode
+// kernel (append, the tag check, the wide pre-pass) use it, so that the SMs
+// they run on are already split for the decode CTAs' shared memory: an SM
+// can change its split only when it is empty, and decode CTAs would
+// otherwise wait there until those kernels' CTAs have exited.
+template <typename K>
+cudaError_t prefer_max_shared(K* kernel);
+
 }  // namespace kvq

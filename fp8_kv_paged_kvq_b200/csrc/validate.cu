@@ -115,19 +115,65 @@ __global__ void __launch_bounds__(kValThreads)
 // waiting while the check runs.  The block-table entries of all requests form
 // one flat index space (request b owns [pre[b], pre[b+1])); CTA g takes the
 // g-th of gridDim.x equal slices, so long and short requests cost alike.
-// Failures go to a per-request word in device memory (the largest
-// INT32_MAX - i over failing entries i, so 0 means none); the last CTA to
-// finish (a ticket that also counts the CTAs that saw a failure) writes every
-// request's mask byte and telemetry and puts the words and the ticket back to
-// 0, reading the words only when some CTA failed.  The words are shared by
-// the library's calls on one device, so these calls must not overlap.
+//
+// Outputs without a combining step.  Before the dependency wait (while the
+// append still runs) CTA 0 writes the result of a clean call: every mask byte
+// 0, every first_bad -1, n_aborted 0, and then publishes that it has done so
+// for this call's epoch.  After the wait a CTA whose entries all pass simply
+// exits, so a clean call ends as soon as its gathers do.  A CTA that finds a
+// failing entry waits until CTA 0 has published for this epoch and then
+// writes over the clean result: mask byte 1, first_bad lowered to the
+// failing index (an unsigned minimum, under which -1 is the largest value),
+// and n_aborted raised by one for the request's first recorded failure.
+//
+// The epoch comes from device memory, so CUDA graph replays of one call get
+// fresh epochs: before its wait every CTA reads the epoch and takes an
+// arrival ticket; the last CTA to arrive puts the ticket back to 0 and
+// advances the epoch for the next call.  These words (and the per-request
+// epochs that dedupe the abort count when first_bad is not requested) are
+// shared by the library's calls on one device, so such calls must not run
+// at the same time.
 // ---------------------------------------------------------------------------
 constexpr int kFlatThreads = 128;
 constexpr int kFlatPer = 8;                 // entries per thread and round
-constexpr int kFlatMaxB = 4096;             // prefix of B + 1 ints in shared memory
+constexpr int kFlatMaxB = 4096;             // prefix of B + 1 ints in (dynamic) shared memory
 
-__device__ int32_t g_val_acc[kFlatMaxB];
-__device__ uint32_t g_val_ticket = 0;       // (CTAs that failed << 16) | CTAs done
+__device__ uint32_t g_val_epoch = 1;        // epoch of the next call (never 0)
+__device__ uint32_t g_val_arrive = 0;       // CTAs of the current call that have read it
+__device__ uint32_t g_val_ready = 0xFFFFFFFFu;   // epoch whose clean result CTA 0 has written
+__device__ uint32_t g_val_seen[kFlatMaxB];  // epoch in which request b was last counted
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
+// Wait (bounded, about one second) until CTA 0 has written this call's clean
+// result.  On a timeout the error word records it and the caller goes on:
+// CTA 0 writes that result before its dependency wait, so it is long done.
+__device__ __forceinline__ void wait_clean_result(uint32_t epoch) {
+  if (ld_acquire_gpu(&g_val_ready) == epoch) return;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_gpu(&g_val_ready) == epoch) return;
+    if ((it & 255u) == 0 && globaltimer_ns() - t0 > 1000000000ull) {
+      atomicOr(&g_error_flags, kErrWaitTimeout);
+      return;
+    }
+  }
+}
 
 __global__ void __maxnreg__(32)
     validate_flat_kernel(const uint32_t* __restrict__ tags, int32_t P,
@@ -138,12 +184,31 @@ __global__ void __maxnreg__(32)
                          int32_t* __restrict__ n_aborted, int32_t* __restrict__ first_bad) {
   // The same programmatic-dependent-launch contract as validate_kernel: the
   // sequence lengths, block table and expected tags are read before the
-  // wait, the live tags after it.
+  // wait, the live tags after it.  In addition the outputs are written
+  // before the wait (CTA 0's clean result).
   pdl_trigger();
-  __shared__ int32_t pre[kFlatMaxB + 1];
+  extern __shared__ int32_t pre[];          // [B + 1]
   __shared__ int32_t warp_sum[kFlatThreads / 32];
-  __shared__ uint32_t ticket;
+  __shared__ uint32_t epoch_sh;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    // the read of the epoch comes before this CTA's arrival (acquire, then
+    // an acquire-release ticket), and the last arrival advances it
+    const uint32_t e = ld_acquire_gpu(&g_val_epoch);
+    if (atom_add_acq_rel_gpu(&g_val_arrive, 1u) == gridDim.x - 1) {
+      g_val_arrive = 0;                     // every CTA of this call has read the epoch
+      st_release_gpu(&g_val_epoch, e + 1u == 0u ? 1u : e + 1u);
+    }
+    epoch_sh = e;
+  }
+  if (blockIdx.x == 0) {
+    for (int b = tid; b < B; b += kFlatThreads) {
+      abort_mask[b] = 0;
+      if (first_bad != nullptr) first_bad[b] = -1;
+    }
+    if (tid == 0 && n_aborted != nullptr) *n_aborted = 0;
+    __threadfence();
+  }
   const int64_t cap = static_cast<int64_t>(max_pages) * ps;
   // pages per request, then an exclusive prefix (each thread a run of requests)
   const int per = (B + kFlatThreads - 1) / kFlatThreads;
@@ -162,7 +227,9 @@ __global__ void __maxnreg__(32)
     if (lane >= o) incl += v;
   }
   if (lane == 31) warp_sum[warp] = incl;
-  __syncthreads();
+  __syncthreads();                          // also: epoch_sh, CTA 0's clean result issued
+  const uint32_t epoch = epoch_sh;
+  if (blockIdx.x == 0 && tid == 0) st_release_gpu(&g_val_ready, epoch);
   int32_t base = incl - run;
   for (int w = 0; w < warp; ++w) base += warp_sum[w];
   for (int b = r0; b < r1; ++b) {
@@ -210,68 +277,45 @@ __global__ void __maxnreg__(32)
     }
   };
   load_round(f0);
-  // The live tags may still change (kvq_append bumps reallocated pages), but
-  // their lines can come into L2 now: the loads after the wait then hit L2
-  // instead of making scattered DRAM reads on the step's critical path.
-#pragma unroll
-  for (int k = 0; k < kFlatPer; ++k)
-    if (page[k] >= 0 && page[k] < P) prefetch_l2(tags + page[k]);
   pdl_wait();
-  int fail = 0;
   for (int32_t r = f0; r < f1; r += kFlatPer * kFlatThreads) {
     if (r != f0) load_round(r);
-    // all of the round's tag loads first (no store between them), failures
-    // as bits; the rare failing entry then goes to its request's word
+    // every live-tag load of the round is issued before any compare; the
+    // loaded tag replaces the page id, which is no longer needed
+    uint32_t inb = 0;
+#pragma unroll
+    for (int k = 0; k < kFlatPer; ++k)
+      if (page[k] >= 0 && page[k] < P) inb |= 1u << k;
+#pragma unroll
+    for (int k = 0; k < kFlatPer; ++k)
+      page[k] = ((inb >> k) & 1u) ? static_cast<int32_t>(ld_global_hint(tags + page[k], keep)) : 0;
     uint32_t bits = 0;
 #pragma unroll
     for (int k = 0; k < kFlatPer; ++k) {
       const int32_t f = r + k * kFlatThreads + tid;
-      const int32_t p = page[k];
-      const bool in = p >= 0 && p < P;
-      const uint32_t live = in ? ld_global_hint(tags + p, keep) : 0u;
-      if (f < f1 && (!in || live != want[k])) bits |= 1u << k;
+      const bool in = (inb >> k) & 1u;
+      if (f < f1 && (!in || static_cast<uint32_t>(page[k]) != want[k])) bits |= 1u << k;
     }
     if (bits != 0) {
+      // rare: overwrite the clean result for the failing requests
+      wait_clean_result(epoch);
 #pragma unroll 1
       for (int k = 0; k < kFlatPer; ++k) {
         if ((bits >> k) & 1u) {
           int32_t b, i;
           locate(r + k * kFlatThreads + tid, 0, b, i);
-          atomicMax(&g_val_acc[b], INT32_MAX - i);
+          abort_mask[b] = 1;
+          bool first;
+          if (first_bad != nullptr)
+            first = atomicMin(reinterpret_cast<uint32_t*>(first_bad) + b,
+                              static_cast<uint32_t>(i)) == 0xFFFFFFFFu;
+          else
+            first = atomicExch(&g_val_seen[b], epoch) != epoch;
+          if (first && n_aborted != nullptr) atomicAdd(n_aborted, 1);
         }
       }
-      fail = 1;
     }
   }
-  if (fail) __threadfence();                // this thread's failure words before the ticket
-  const int any = __syncthreads_or(fail);
-  if (tid == 0) {
-    ticket = atomicAdd(&g_val_ticket, 1u + (any ? 0x10000u : 0u)) + (any ? 0x10000u : 0u);
-  }
-  __syncthreads();
-  const uint32_t t = ticket;
-  if ((t & 0xFFFFu) != gridDim.x - 1) return;
-  // last CTA: every other CTA's failure words are visible
-  __threadfence();
-  const bool some = (t >> 16) != 0;
-  int32_t cnt = 0;
-  for (int b = tid; b < B; b += kFlatThreads) {
-    const int32_t v = some ? atomicExch(&g_val_acc[b], 0) : 0;
-    abort_mask[b] = v != 0 ? 1 : 0;
-    if (first_bad != nullptr) first_bad[b] = v != 0 ? INT32_MAX - v : -1;
-    cnt += v != 0 ? 1 : 0;
-  }
-  if (n_aborted != nullptr) {
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (lane == 0) warp_sum[warp] = cnt;
-    __syncthreads();
-    if (tid == 0) {
-      int32_t total = 0;
-      for (int w = 0; w < kFlatThreads / 32; ++w) total += warp_sum[w];
-      *n_aborted = total;
-    }
-  }
-  if (tid == 0) g_val_ticket = 0;
 }
 
 cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* block_table,
@@ -298,9 +342,7 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
         if (e != cudaSuccess) return e;
         // keep the SM's shared memory at its largest split while this runs,
         // so the decode CTAs (about 100 KB each) fit beside it
-        e = cudaFuncSetAttribute(validate_flat_kernel,
-                                 cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
+        e = prefer_max_shared(validate_flat_kernel);
         if (e != cudaSuccess) return e;
         sms_of[dev] = n;
       }
@@ -314,6 +356,7 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kFlatThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(B + 1) * sizeof(int32_t);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -330,6 +373,10 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
   int C = (max_pages + kPerCta - 1) / kPerCta;
   C = C < 1 ? 1 : (C > kMaxCluster ? kMaxCluster : C);
   if (static_cast<int64_t>(B) * C > 0x7fffffff) return cudaErrorInvalidValue;
+  {
+    const cudaError_t e = prefer_max_shared(validate_kernel);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(B * C));
   cfg.blockDim = dim3(kValThreads);

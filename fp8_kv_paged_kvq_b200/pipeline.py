@@ -276,6 +276,9 @@ class DecodeLoop:
             if self.detailed[i]:
                 gs = []
                 for f in parts:
+                    if f is self._validate and k == NOCHECK:
+                        gs.append(None)              # nothing to run between the events
+                        continue
                     g = torch.cuda.CUDAGraph()
                     with torch.cuda.graph(g, stream=stream):
                         f(i, k, stream)
@@ -302,7 +305,8 @@ class DecodeLoop:
             for j, g in enumerate(gs):
                 if events is not None:
                     events[j].record(stream)
-                g.replay()
+                if g is not None:
+                    g.replay()
             if events is not None:
                 events[len(gs)].record(stream)
 

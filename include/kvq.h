@@ -168,11 +168,15 @@ kvq_status kvq_append(const kvq_cache* cache, const void* k_new, const void* v_n
  * Batches of up to 4,096 requests (and B * max_pages < 2^31) run as one CTA
  * of 128 threads per SM over all requests' entries, small enough to share
  * each SM with the decode launch that follows, whose CTAs then start while
- * the check runs.  Its CTAs combine failures through a small accumulator in
- * the library's device memory, which returns to zero at the end of each
- * call: on one device, such calls must not run at the same time (on
- * different streams).  Larger batches use one cluster of up to 8 CTAs per
- * request and have no such restriction.
+ * the check runs.  This form also writes the result of a clean check
+ * (mask 0, first_bad -1, n_aborted 0) while the previous kernel may still
+ * run, and only failing requests are written after it: that kernel must not
+ * read or write abort_mask, n_aborted or first_bad either (kvq_append never
+ * does).  Its CTAs share a few words of the library's device memory (a call
+ * epoch, an arrival count, per-request epochs for the abort count): on one
+ * device, such calls must not run at the same time (on different streams).
+ * Larger batches use one cluster of up to 8 CTAs per request and have no
+ * such restriction.
  */
 kvq_status kvq_validate(const uint32_t* page_tags, int32_t num_pages, const int32_t* block_table,
                         const uint32_t* expected_tags, const int32_t* seq_lens,
@@ -222,7 +226,11 @@ size_t kvq_decode_workspace_size(const kvq_cache* cache, int32_t B, int32_t num_
  * rounded at the E4M3 step 2^-9), and the E4M3 NaN
  * codes 0x7F / 0xFF, which kvq_append never writes, read as +-480 there.
  * The kernels are launched as programmatic dependents of the previous work
- * on the stream and wait for it before reading any argument.
+ * on the stream.  The 8-head kernel reads seq_lens and block_table to plan
+ * its split while that work may still run (the kernel launched just before
+ * must not write them; kvq_validate and kvq_append never do) and everything
+ * else, the abort mask included, after it has finished; the wide kernels
+ * wait before reading any argument.
  */
 kvq_status kvq_decode(const kvq_cache* cache, const void* q, int32_t num_q_heads,
                       const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,
@@ -286,9 +294,12 @@ kvq_status kvq_e4m3_quantize_bits(uint32_t start, uint32_t count, float scale, u
 
 /*
  * Reads and clears the library's device-side error word on the current
- * device (synchronous).  Bit 0: a pipeline wait in a decode kernel gave up
- * after its time limit (about one second) and the kernel returned early, so
- * that launch's outputs are invalid.  *flags_host receives the word.
+ * device (synchronous).  Bit 0: a bounded wait gave up after its time limit
+ * (about one second): a pipeline wait in a decode kernel (the kernel returned
+ * early, so that launch's outputs are invalid), or, in kvq_validate, a
+ * failing CTA's wait for the clean result of the same call (the mask bytes
+ * written after it may then be overwritten by that late clean result, so
+ * the call's outputs are invalid).  *flags_host receives the word.
  */
 kvq_status kvq_device_error(uint32_t* flags_host);
 

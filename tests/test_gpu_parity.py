@@ -298,6 +298,73 @@ def test_validate_batch_sizes_and_reset(B):
         assert int(n_ab.item()) == int(ref.sum())
 
 
+@pytest.mark.parametrize("with_first_bad", [False, True])
+def test_validate_graph_replays_with_changing_tags(with_first_bad):
+    """One kvq_validate call captured in a CUDA graph and replayed with the
+    expected tags changed between replays (stale entries in different
+    requests, then none, then again): each replay's mask, abort count and
+    first failing index equal the oracle's, so nothing of one replay's
+    outcome leaks into the next."""
+    r = np.random.default_rng(40)
+    P, B, maxp, ps = 3000, 64, 40, 16
+    tags = r.integers(0, 1 << 32, P, dtype=np.uint64).astype(np.uint32)
+    bt = r.integers(0, P, (B, maxp)).astype(np.int32)
+    lens = r.integers(0, maxp * ps + 1, B).astype(np.int32)
+    clean = tags[bt].copy()
+    dev = lambda a: torch.from_numpy(a).cuda()
+    d_tags, d_bt, d_lens = dev(tags.view(np.int32)), dev(bt), dev(lens)
+    d_exp = dev(clean.view(np.int32))
+    mask = torch.empty(B, dtype=torch.uint8, device="cuda")
+    n_ab = torch.full((1,), 77, dtype=torch.int32, device="cuda")
+    first = torch.full((B,), 5, dtype=torch.int32, device="cuda") if with_first_bad else None
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        kvq.validate(d_tags, d_bt, d_exp, d_lens, ps, mask, stream, n_aborted=n_ab, first_bad=first)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            kvq.validate(d_tags, d_bt, d_exp, d_lens, ps, mask, stream, n_aborted=n_ab,
+                         first_bad=first)
+    for trial in range(12):
+        exp = clean.copy()
+        if trial % 3 != 1:
+            hit = r.integers(0, B, int(r.integers(1, 6)))
+            exp[hit, r.integers(0, maxp, hit.size)] ^= 1
+        d_exp.copy_(torch.from_numpy(exp.view(np.int32)))
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        ref, ref_first = oracle.validate(tags, bt, exp, lens, ps, first_bad=True)
+        assert np.array_equal(mask.cpu().numpy(), ref), trial
+        assert int(n_ab.item()) == int(ref.sum()), trial
+        if with_first_bad:
+            assert np.array_equal(first.cpu().numpy(), ref_first), trial
+    assert kvq.device_error() == 0
+
+
+def test_validate_abort_count_without_first_bad():
+    """The abort count alone (no per-request index requested), over calls in
+    a row where the same requests fail again: each call counts each aborted
+    request once."""
+    r = np.random.default_rng(41)
+    for trial in range(10):
+        P, B, maxp, ps = 2000, int(r.integers(1, 300)), int(r.integers(1, 200)), 16
+        tags = r.integers(0, 1 << 32, P, dtype=np.uint64).astype(np.uint32)
+        bt = r.integers(-1, P + 1, (B, maxp)).astype(np.int32)
+        lens = r.integers(0, maxp * ps + 1, B).astype(np.int32)
+        exp = tags[np.clip(bt, 0, P - 1)].copy()
+        exp[r.random((B, maxp)) < 0.01] ^= 1
+        dev = lambda a: torch.from_numpy(a).cuda()
+        for _ in range(2):
+            n_ab = torch.full((1,), -3, dtype=torch.int32, device="cuda")
+            got = kvq.validate(dev(tags.view(np.int32)), dev(bt), dev(exp.view(np.int32)),
+                               dev(lens), ps, n_aborted=n_ab)
+            ref = oracle.validate(tags, bt, exp, lens, ps)
+            assert np.array_equal(got.cpu().numpy(), ref), trial
+            assert int(n_ab.item()) == int(ref.sum()), trial
+    assert kvq.device_error() == 0
+
+
 def test_tag_bump_matches_oracle():
     P = 50
     tags = np.random.default_rng(1).integers(0, 2**32, P, dtype=np.uint64).astype(np.uint32)
