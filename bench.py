@@ -636,11 +636,15 @@ def run_long(args, rank, world, local, dev):
     torch.cuda.synchronize()
     loop.snapshot_tags()
     stream = torch.cuda.Stream(device=dev)
-    # kinds cycle stale / clean / no check; every other cycle of three steps
-    # runs each call as its own graph with events between them (the decode
-    # call's time), the others as one graph per step with events only at the
-    # step's boundaries (the step times)
-    kinds = [(STALE, CLEAN, NOCHECK)[i % 3] for i in range(n)]
+    # kinds cycle in twelve steps: stale / clean / no check, then stale / no
+    # check / clean, so that clean and unchecked steps follow the same mix of
+    # neighbours; every other cycle of three steps runs each call as its own
+    # graph with events between them (the decode call's time), the others as
+    # one graph per step with events only at the step's boundaries (the step
+    # times)
+    order = (STALE, CLEAN, NOCHECK, STALE, CLEAN, NOCHECK,
+             STALE, NOCHECK, CLEAN, STALE, NOCHECK, CLEAN)
+    kinds = [order[i % 12] for i in range(n)]
     detailed = [(i // 3) % 2 == 1 for i in range(n)]
     loop.capture(stream, kinds, detailed)
     row = spec.num_kv_heads * (spec.head_dim_k + spec.head_dim_v)
@@ -715,7 +719,8 @@ def run_long(args, rank, world, local, dev):
         "config": {"workload": workload_desc("long"),
                    "loop": f"{n} decode steps per pass: append 1 token/seq with page "
                            "reallocation + tag bump, then the tag check, then decode; steps "
-                           "cycle check with 0.01% stale tags / clean check / no check",
+                           "cycle check with 0.01% stale tags / clean check / no check (and "
+                           "stale / no check / clean)",
                    "steps_and_warmup": f"passes over the {n}-step loop (each pass resets the "
                                        "live tags and repeats the same tag history)",
                    "ms_per_step": "one decode step (append + validate + decode), mean over "

@@ -191,24 +191,6 @@ __global__ void __maxnreg__(32)
   __shared__ int32_t warp_sum[kFlatThreads / 32];
   __shared__ uint32_t epoch_sh;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) {
-    // the read of the epoch comes before this CTA's arrival (acquire, then
-    // an acquire-release ticket), and the last arrival advances it
-    const uint32_t e = ld_acquire_gpu(&g_val_epoch);
-    if (atom_add_acq_rel_gpu(&g_val_arrive, 1u) == gridDim.x - 1) {
-      g_val_arrive = 0;                     // every CTA of this call has read the epoch
-      st_release_gpu(&g_val_epoch, e + 1u == 0u ? 1u : e + 1u);
-    }
-    epoch_sh = e;
-  }
-  if (blockIdx.x == 0) {
-    for (int b = tid; b < B; b += kFlatThreads) {
-      abort_mask[b] = 0;
-      if (first_bad != nullptr) first_bad[b] = -1;
-    }
-    if (tid == 0 && n_aborted != nullptr) *n_aborted = 0;
-    __threadfence();
-  }
   const int64_t cap = static_cast<int64_t>(max_pages) * ps;
   // pages per request, then an exclusive prefix (each thread a run of requests)
   const int per = (B + kFlatThreads - 1) / kFlatThreads;
@@ -227,9 +209,7 @@ __global__ void __maxnreg__(32)
     if (lane >= o) incl += v;
   }
   if (lane == 31) warp_sum[warp] = incl;
-  __syncthreads();                          // also: epoch_sh, CTA 0's clean result issued
-  const uint32_t epoch = epoch_sh;
-  if (blockIdx.x == 0 && tid == 0) st_release_gpu(&g_val_ready, epoch);
+  __syncthreads();
   int32_t base = incl - run;
   for (int w = 0; w < warp; ++w) base += warp_sum[w];
   for (int b = r0; b < r1; ++b) {
@@ -277,6 +257,28 @@ __global__ void __maxnreg__(32)
     }
   };
   load_round(f0);
+  // With the first entries' loads in flight: the call's epoch (its read comes
+  // before this CTA's arrival, an acquire-release ticket; the last arrival
+  // advances it) and, in CTA 0, the clean result, published for the epoch.
+  if (tid == 0) {
+    const uint32_t e = ld_acquire_gpu(&g_val_epoch);
+    if (atom_add_acq_rel_gpu(&g_val_arrive, 1u) == gridDim.x - 1) {
+      g_val_arrive = 0;                     // every CTA of this call has read the epoch
+      st_release_gpu(&g_val_epoch, e + 1u == 0u ? 1u : e + 1u);
+    }
+    epoch_sh = e;
+  }
+  if (blockIdx.x == 0) {
+    for (int b = tid; b < B; b += kFlatThreads) {
+      abort_mask[b] = 0;
+      if (first_bad != nullptr) first_bad[b] = -1;
+    }
+    if (tid == 0 && n_aborted != nullptr) *n_aborted = 0;
+    __threadfence();
+  }
+  __syncthreads();                          // epoch_sh; CTA 0's clean result written
+  const uint32_t epoch = epoch_sh;
+  if (blockIdx.x == 0 && tid == 0) st_release_gpu(&g_val_ready, epoch);
   pdl_wait();
   for (int32_t r = f0; r < f1; r += kFlatPer * kFlatThreads) {
     if (r != f0) load_round(r);
@@ -348,11 +350,16 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
       }
       sms = sms_of[dev];
     }
-    // at most one CTA per SM, and no more than B * max_pages entries need:
-    // one round of kFlatPer loads per thread either way up to 148K entries
+    // No more CTAs than B * max_pages entries need, and at most 7/8 of the
+    // SMs: the append kernel's few CTAs occupy some SMs when this grid is
+    // placed, and a full grid then doubles up on others, where two of these
+    // CTAs leave no room for the second decode CTA until one exits.  One
+    // round of kFlatPer loads per thread covers 1,024 entries per CTA
+    // (133K entries on a 148-SM B200).
     const int64_t per_cta = static_cast<int64_t>(kFlatThreads) * kFlatPer;
     const int64_t want = (static_cast<int64_t>(B) * max_pages + per_cta - 1) / per_cta;
-    const int grid = static_cast<int>(want < 1 ? 1 : (want < sms ? want : sms));
+    const int cap = sms - sms / 8 > 0 ? sms - sms / 8 : 1;
+    const int grid = static_cast<int>(want < 1 ? 1 : (want < cap ? want : cap));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kFlatThreads);
