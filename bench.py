@@ -84,23 +84,36 @@ def parse(argv=None):
     return ap.parse_args(argv)
 
 
-def measured_traffic(workload, seqs):
-    """DRAM bytes per decode launch from the committed ncu record, or None when
-    the kernel source changed since the capture or the workload differs."""
+def measured_traffic(kernel, units):
+    """DRAM bytes of one decode launch from the committed ncu record (bytes per
+    unit x the launch's units), or None when the kernel source changed since
+    the capture.  Records without a per-unit figure give their per-launch
+    bytes for the workload they were taken on."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if seqs or not os.path.exists(p):
+    if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f)
-    for r in rec.values():
+    for name, r in rec.items():
+        if not name.startswith(kernel):
+            continue
         src = os.path.join(ROOT, r["source"])
-        if not os.path.exists(src) or r.get("workload") != workload:
+        if not os.path.exists(src):
             continue
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if h == r["source_sha256_prefix"]:
-            return r["dram_bytes_per_launch"]
+        if h != r["source_sha256_prefix"]:
+            return None
+        if "dram_bytes_per_unit" in r:
+            return r["dram_bytes_per_unit"] * units
+        return None
     return None
+
+
+def gqa_units(spec, seq_lens):
+    """Work units of the 8-head decode kernel: 16-token tiles per (sequence, KV head)."""
+    lens = np.asarray(seq_lens, np.int64)
+    return int(((lens + 15) // 16).sum()) * spec.num_kv_heads
 
 
 def _peaks_file():
@@ -501,7 +514,8 @@ def measure_batch(name, args, dev, stream, world, e2e=True, bf16=True, cpu=True)
            "ms_per_step": st, "ms_per_step_without_validation": sn, "ms_decode_call": sd,
            "validate_overhead_pct": 100.0 * (st["mean"] - sn["mean"]) / sn["mean"],
            "roofline": decode_roofline(s, lens, max_over_ranks(sd["mean"], world),
-                                       measured_traffic(name, args.seqs)),
+                                       None if is_wide(s) else
+                                       measured_traffic("gqa_decode_kernel", gqa_units(s, lens))),
            "timing": "CUDA graph replays, events around every replay, "
                      f">= {args.min_seconds} s each; inputs exceed L2"}
     assert_no_device_error()
@@ -705,10 +719,14 @@ def run_long(args, rank, world, local, dev):
     # detailed steps: algorithmic bytes / time, summed over those steps
     dec_ms = m(t_dec[dclean].sum()) / dclean.sum()
     dec_bytes = alg_dec[idx[dclean]].mean()
-    roof = decode_roofline(spec, lens[n // 2], dec_ms, measured_traffic("long", 0),
-                           alg_bytes=dec_bytes)
+    dec_units = np.mean([gqa_units(spec, [lens[i, b] for b in range(spec.B)
+                                          if b not in aborted[i]]) for i in idx[dclean]])
+    roof = decode_roofline(spec, lens[n // 2], dec_ms,
+                           measured_traffic("gqa_decode_kernel", dec_units), alg_bytes=dec_bytes)
     roof["note"] = ("decode call between events inside the clean steps of the timed passes; "
-                    "algorithmic bytes and time averaged over those steps")
+                    "algorithmic bytes and time averaged over those steps; traffic = DRAM "
+                    "bytes per 16-token tile from an ncu capture of the 8-head kernel on 8 "
+                    "of the gqa batch's sequences, times the tiles of the average step")
     hbm, _ = peaks()
     launches = sum(3 if k == NOCHECK else 4 for k in kinds) * args.steps
     line = {

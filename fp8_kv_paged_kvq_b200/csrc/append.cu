@@ -439,8 +439,6 @@ cudaError_t launch_append(const CacheView& c, const uint16_t* k_new, const uint1
   a.token_blocks = static_cast<int32_t>((warps + kAppendWarps - 1) / kAppendWarps);
   const int32_t blocks = a.token_blocks + (n_realloc > 0 ? 1 : 0);
   if (blocks == 0) return cudaSuccess;
-  const cudaError_t e = prefer_max_shared(append_kernel);
-  if (e != cudaSuccess) return e;
   append_kernel<<<blocks, kAppendWarps * 32, 0, stream>>>(a);
   return cudaGetLastError();
 }

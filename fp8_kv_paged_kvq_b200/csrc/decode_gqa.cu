@@ -628,8 +628,8 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
 // [c*U/N, (c+1)*U/N), so unit u belongs to CTA ((u+1)*N - 1) / U and the
 // pieces of a segment with units [S, E) are exactly the CTAs cs..ce that own
 // S and E - 1, every one of them non-empty.  With up to kCombFast pieces
-// each thread loads its outputs' partials from every piece in one round and
-// merges them itself: out = sum_k exp(lse_k - M) / L * o_k with M the
+// each thread loads its four outputs' partials from every piece in one round
+// and merges them itself: out = sum_k exp(lse_k - M) / L * o_k with M the
 // largest lse_k and L the sum of exp(lse_k - M).  With more pieces, warp w
 // first forms M and L for its heads, and the block then takes the pieces in
 // chunks of kCombChunk whose weights it stages in shared memory.
@@ -643,11 +643,10 @@ struct CombineParams {
   float* lse;
 };
 
-constexpr int kCombThreads = 256;
 constexpr int kCombHeads = 32;        // heads per block at most
 constexpr int kCombChunk = 64;        // pieces whose weights are staged at once
 constexpr int kCombOutputs = 4096;    // outputs per block (heads_per_block * Dv) at most
-constexpr int kCombPerThread = kCombOutputs / 4 / kCombThreads;   // float4 outputs per thread
+constexpr int kCombMaxThreads = kCombOutputs / 4;   // one group of four outputs per thread
 constexpr int kCombFast = 4;          // pieces merged from registers in one round of loads
 
 // CTA of a launch with N working CTAs over U units that owns unit u.
@@ -655,7 +654,10 @@ __device__ __forceinline__ int64_t owner_cta(int64_t u, int64_t N, int64_t U) {
   return ((u + 1) * N - 1) / U;
 }
 
-__global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const CombineParams p) {
+// One thread per group of four consecutive output dims of the block's heads
+// (blockDim = heads_per_block * Dv / 4, at most kCombMaxThreads), so the
+// blocks are small and all of a launch's blocks are resident at once.
+__global__ void __launch_bounds__(kCombMaxThreads) lse_combine_kernel(const CombineParams p) {
   pdl_wait();                                    // the decode kernel has finished
   const int32_t seg = blockIdx.x;
   const int32_t b = seg / p.Hkv, h = seg - b * p.Hkv;
@@ -665,11 +667,26 @@ __global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const Combine
   const int32_t tiles_b = (p.ws_pre[b + 1] - p.ws_pre[b]) / p.Hkv;
   float* out = p.out + (static_cast<int64_t>(b) * p.Hq + h * p.G + h0) * p.Dv;
   float* lse = p.lse ? p.lse + static_cast<int64_t>(b) * p.Hq + h * p.G + h0 : nullptr;
-  const int n_out = nh * p.Dv;
+  const int dq = p.Dv >> 2;                     // outputs in groups of four dims
+  const int n4 = nh * dq;
+  const int i4 = threadIdx.x;                   // this thread's group
+  const bool mine = i4 < n4;
+  const int hh = mine ? i4 / dq : 0, d = mine ? (i4 - hh * dq) * 4 : 0;
+  const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+  auto store = [&](const float4& acc) {
+    float* dst = out + hh * p.Dv + d;
+    if (vec_out) {
+      *reinterpret_cast<float4*>(dst) = acc;
+    } else {
+      dst[0] = acc.x;
+      dst[1] = acc.y;
+      dst[2] = acc.z;
+      dst[3] = acc.w;
+    }
+  };
   if (tiles_b == 0) {
-    for (int idx = threadIdx.x; idx < n_out; idx += blockDim.x) out[idx] = 0.0f;
-    if (lse)
-      for (int hh = threadIdx.x; hh < nh; hh += blockDim.x) lse[hh] = -__int_as_float(0x7f800000);
+    if (mine) store(make_float4(0.f, 0.f, 0.f, 0.f));
+    if (lse && mine && d == 0) lse[hh] = -__int_as_float(0x7f800000);
     return;
   }
   // U >= tiles_b > 0 here
@@ -678,80 +695,61 @@ __global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const Combine
   const int64_t cs = owner_cta(S, N, U);
   const int np = static_cast<int>(owner_cta(E - 1, N, U) - cs + 1);
   const int64_t slot0 = cs + seg;               // slot of piece k: slot0 + k
-  const int dq = p.Dv >> 2;                     // outputs in groups of four dims
-  const int n4 = nh * dq;
-  const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
   if (np <= kCombFast) {
-    // Few pieces: thread t loads, in one round, the partial outputs of its
-    // groups t, t + kCombThreads, ... and the partial lse of their heads
-    // from every piece, and merges them on its own.
-    float4 o[kCombPerThread][kCombFast];
-    float a[kCombPerThread][kCombFast];
+    // few pieces: one round of loads of this group's partial outputs and its
+    // head's partial lse from every piece, merged in registers
+    if (!mine) return;
+    float4 o[kCombFast];
+    float a[kCombFast];
 #pragma unroll
-    for (int r = 0; r < kCombPerThread; ++r) {
-      const int i4 = threadIdx.x + r * kCombThreads;
-      const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
+    for (int k = 0; k < kCombFast; ++k) {
+      if (k < np) {
+        const int64_t row = (slot0 + k) * p.G + h0 + hh;
+        o[k] = *reinterpret_cast<const float4*>(p.ws_o + row * p.Dv + d);
+        a[k] = p.ws_lse[row];
+      }
+    }
+    float4 acc = o[0];                           // a single piece is copied bit for bit
+    float lse_h = a[0];
+    if (np > 1) {
+      float M = a[0];
+#pragma unroll
+      for (int k = 1; k < kCombFast; ++k)
+        if (k < np) M = fmaxf(M, a[k]);
+      float L = 0.0f, w[kCombFast];
 #pragma unroll
       for (int k = 0; k < kCombFast; ++k) {
-        if (i4 < n4 && k < np) {
-          const int64_t row = (slot0 + k) * p.G + h0 + hh;
-          o[r][k] = *reinterpret_cast<const float4*>(p.ws_o + row * p.Dv + d);
-          a[r][k] = p.ws_lse[row];
+        w[k] = k < np ? __expf(a[k] - M) : 0.0f;
+        L += w[k];
+      }
+      const float inv = 1.0f / L;
+      acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < kCombFast; ++k) {
+        if (k < np) {
+          const float wk = w[k] * inv;
+          acc.x += wk * o[k].x;
+          acc.y += wk * o[k].y;
+          acc.z += wk * o[k].z;
+          acc.w += wk * o[k].w;
         }
       }
+      lse_h = M + __logf(L);
     }
-#pragma unroll
-    for (int r = 0; r < kCombPerThread; ++r) {
-      const int i4 = threadIdx.x + r * kCombThreads;
-      if (i4 >= n4) continue;
-      const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
-      float4 acc = o[r][0];                      // a single piece is copied bit for bit
-      float lse_h = a[r][0];
-      if (np > 1) {
-        float M = a[r][0];
-#pragma unroll
-        for (int k = 1; k < kCombFast; ++k)
-          if (k < np) M = fmaxf(M, a[r][k]);
-        float L = 0.0f, w[kCombFast];
-#pragma unroll
-        for (int k = 0; k < kCombFast; ++k) {
-          w[k] = k < np ? __expf(a[r][k] - M) : 0.0f;
-          L += w[k];
-        }
-        const float inv = 1.0f / L;
-        acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < kCombFast; ++k) {
-          if (k < np) {
-            const float wk = w[k] * inv;
-            acc.x += wk * o[r][k].x;
-            acc.y += wk * o[r][k].y;
-            acc.z += wk * o[r][k].z;
-            acc.w += wk * o[r][k].w;
-          }
-        }
-        lse_h = M + __logf(L);
-      }
-      if (lse && d == 0) lse[hh] = lse_h;
-      float* dst = out + hh * p.Dv + d;
-      if (vec_out) {
-        *reinterpret_cast<float4*>(dst) = acc;
-      } else {
-        dst[0] = acc.x;
-        dst[1] = acc.y;
-        dst[2] = acc.z;
-        dst[3] = acc.w;
-      }
-    }
+    if (lse && d == 0) lse[hh] = lse_h;
+    store(acc);
     return;
   }
+  // many pieces: warp w forms the maximum M and the sum L for heads w,
+  // w + warps, ...; then the block takes the pieces in chunks whose weights
+  // exp(lse_k - M) / L it stages in shared memory
   __shared__ float m_sh[kCombHeads], inv_sh[kCombHeads];
   __shared__ float wts[kCombHeads][kCombChunk];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
   const float kNegInf = -__int_as_float(0x7f800000);
-  for (int hh = warp; hh < nh; hh += kCombThreads / 32) {
-    const int head = h0 + hh;
-    const float* l = p.ws_lse + slot0 * p.G + head;   // piece k at l[k * G]
+  for (int x = warp; x < nh; x += nwarps) {
+    const float* l = p.ws_lse + slot0 * p.G + h0 + x;   // piece k at l[k * G]
     float M = kNegInf;
     for (int k = lane; k < np; k += 32) M = fmaxf(M, l[static_cast<int64_t>(k) * p.G]);
 #pragma unroll
@@ -761,62 +759,37 @@ __global__ void __launch_bounds__(kCombThreads) lse_combine_kernel(const Combine
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     if (lane == 0) {
-      m_sh[hh] = M;
-      inv_sh[hh] = 1.0f / L;
-      if (lse) lse[hh] = M + __logf(L);
+      m_sh[x] = M;
+      inv_sh[x] = 1.0f / L;
+      if (lse) lse[x] = M + __logf(L);
     }
   }
-  // many pieces: thread t holds groups t, t + kCombThreads, ... and the
-  // pieces come in chunks whose weights are staged in shared memory
-  float4 acc[kCombPerThread];
-#pragma unroll
-  for (int r = 0; r < kCombPerThread; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-  {
-    __syncthreads();                             // m_sh, inv_sh
-    for (int base = 0; base < np; base += kCombChunk) {
-      const int nk = min(kCombChunk, np - base);
-      for (int idx = threadIdx.x; idx < nh * nk; idx += kCombThreads) {
-        const int hh = idx / nk, k = idx - hh * nk;
-        const float a = p.ws_lse[(slot0 + base + k) * p.G + h0 + hh];
-        wts[hh][k] = __expf(a - m_sh[hh]) * inv_sh[hh];
-      }
-      __syncthreads();
-#pragma unroll
-      for (int r = 0; r < kCombPerThread; ++r) {
-        const int i4 = threadIdx.x + r * kCombThreads;
-        if (i4 < n4) {
-          const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
-          const float* o = p.ws_o + ((slot0 + base) * p.G + h0 + hh) * p.Dv + d;
-          const int64_t stride = static_cast<int64_t>(p.G) * p.Dv;   // next piece
+  __syncthreads();                               // m_sh, inv_sh
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int base = 0; base < np; base += kCombChunk) {
+    const int nk = min(kCombChunk, np - base);
+    for (int idx = threadIdx.x; idx < nh * nk; idx += blockDim.x) {
+      const int x = idx / nk, k = idx - x * nk;
+      const float a = p.ws_lse[(slot0 + base + k) * p.G + h0 + x];
+      wts[x][k] = __expf(a - m_sh[x]) * inv_sh[x];
+    }
+    __syncthreads();
+    if (mine) {
+      const float* o = p.ws_o + ((slot0 + base) * p.G + h0 + hh) * p.Dv + d;
+      const int64_t stride = static_cast<int64_t>(p.G) * p.Dv;   // next piece
 #pragma unroll 4
-          for (int k = 0; k < nk; ++k) {
-            const float4 v = *reinterpret_cast<const float4*>(o + k * stride);
-            const float w = wts[hh][k];
-            acc[r].x += w * v.x;
-            acc[r].y += w * v.y;
-            acc[r].z += w * v.z;
-            acc[r].w += w * v.w;
-          }
-        }
+      for (int k = 0; k < nk; ++k) {
+        const float4 v = *reinterpret_cast<const float4*>(o + k * stride);
+        const float w = wts[hh][k];
+        acc.x += w * v.x;
+        acc.y += w * v.y;
+        acc.z += w * v.z;
+        acc.w += w * v.w;
       }
-      __syncthreads();                           // wts reused by the next chunk
     }
+    __syncthreads();                             // wts reused by the next chunk
   }
-#pragma unroll
-  for (int r = 0; r < kCombPerThread; ++r) {
-    const int i4 = threadIdx.x + r * kCombThreads;
-    if (i4 >= n4) continue;
-    const int hh = i4 / dq, d = (i4 - hh * dq) * 4;
-    float* dst = out + hh * p.Dv + d;
-    if (vec_out) {
-      *reinterpret_cast<float4*>(dst) = acc[r];
-    } else {
-      dst[0] = acc[r].x;
-      dst[1] = acc[r].y;
-      dst[2] = acc[r].z;
-      dst[3] = acc[r].w;
-    }
-  }
+  if (mine) store(acc);
 }
 
 // ---------------------------------------------------------------------------
@@ -837,13 +810,16 @@ cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const
   cp.num_ctas = num_ctas;
   cp.out = out;
   cp.lse = lse;
-  int hpb = kCombOutputs / (Dv > 0 ? Dv : 1);
-  hpb = hpb < 1 ? 1 : (hpb > kCombHeads ? kCombHeads : hpb);
-  cp.heads_per_block = hpb;
   if (Dv % 4 != 0 || Dv > kCombOutputs) return cudaErrorInvalidValue;
+  int hpb = kCombOutputs / Dv;
+  hpb = hpb < 1 ? 1 : (hpb > kCombHeads ? kCombHeads : hpb);
+  hpb = hpb > G ? G : hpb;
+  cp.heads_per_block = hpb;
+  // one thread per four outputs of the block, in whole warps
+  const int threads = (hpb * (Dv / 4) + 31) / 32 * 32;
   const dim3 grid(static_cast<unsigned>(B * Hkv), static_cast<unsigned>((G + hpb - 1) / hpb));
   if (B * Hkv == 0) return cudaSuccess;
-  return launch_pdl(lse_combine_kernel, grid, dim3(kCombThreads), 0, stream, cp);
+  return launch_pdl(lse_combine_kernel, grid, dim3(threads), 0, stream, cp);
 }
 
 // Opt the kernel into the largest dynamic shared memory it can ask for, once

@@ -36,11 +36,12 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
 cudaError_t read_and_clear_error_flags(uint32_t* flags);
 
 // Ask for the largest shared-memory carveout for `kernel` on the current
-// device (once per device).  The small kernels launched just before a decode
-// kernel (append, the tag check, the wide pre-pass) use it, so that the SMs
-// they run on are already split for the decode CTAs' shared memory: an SM
-// can change its split only when it is empty, and decode CTAs would
-// otherwise wait there until those kernels' CTAs have exited.
+// device (once per device).  The tag check and the wide pre-pass, which run
+// beside the decode CTAs that follow them, use it, so that the SMs they
+// occupy are already split for the decode CTAs' shared memory (an SM changes
+// its split only when it is empty).  The append kernel keeps the default: its
+// streaming loads want L1, and its CTAs exit before a decode launch that
+// follows a tag check needs their SMs.
 template <typename K>
 cudaError_t prefer_max_shared(K* kernel);
 

@@ -275,8 +275,8 @@ class DecodeLoop:
             k = self.kinds[i]
             if self.detailed[i]:
                 gs = []
-                for f in parts:
-                    if f is self._validate and k == NOCHECK:
+                for part, f in enumerate(parts):
+                    if part == 1 and k == NOCHECK:
                         gs.append(None)              # nothing to run between the events
                         continue
                     g = torch.cuda.CUDAGraph()

@@ -1,10 +1,10 @@
 """The append kernel's quantize step reaches RN(v / s) without a division per
 value (Markstein's correction step; see the quotient notes in csrc/append.cu).
 This pins the arithmetic fact it relies on, in IEEE binary32 with
-fused multiply-add on the host, for every bf16 significand against float
-significands of the scale: a stride through all 2^23 of them plus the
-patterns that stress a reciprocal (all-ones, zero, the repeating 1/7 of
-amax / 448 scales).  A negative control shows the check can fail."""
+fused multiply-add on the host, for every bf16 significand against every
+float significand of the scale (all 2^23), plus the patterns that stress a
+reciprocal (all-ones, zero, the repeating 1/7 of amax / 448 scales).  A
+negative control shows the check can fail."""
 import os
 import re
 import subprocess
@@ -32,8 +32,8 @@ def run(exe, first, count, stride, control=False):
 
 
 def test_corrected_product_is_the_ieee_quotient(checker):
-    n, bad = run(checker, 0, 1 << 16, 127)                 # 65,536 significands across [1, 2)
-    assert n == 128 << 16 and bad == 0
+    n, bad = run(checker, 0, 1 << 23, 1)                   # every float significand in [1, 2)
+    assert n == 128 << 23 and bad == 0
     for m in (0x7FFFFF, 0x000000, 0x000001, 0x7FFFFE, 0x492492, 0x36DB6D, 0x5B6DB7, 0x12492):
         assert run(checker, m, 1, 1) == (128, 0)
 
