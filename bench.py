@@ -472,11 +472,16 @@ def workload_desc(name, seqs=0):
 # ---------------------------------------------------------------------------
 # one decode batch (gqa, ragged, wide): the step, the decode call, e2e
 # ---------------------------------------------------------------------------
+REPS = 8   # calls per CUDA graph in the single-batch measurements
+
+
 def measure_batch(name, args, dev, stream, world, e2e=True, bf16=True, cpu=True):
     """Step and decode-call statistics of one decode batch.  The step
-    (append -> validate -> decode) and the decode call are CUDA graphs, each
-    replayed with events around every replay until args.min_seconds of device
-    time; the inputs exceed L2, so no flush is needed between replays."""
+    (append -> validate -> decode) and the decode call are each captured
+    REPS times back to back in one CUDA graph, replayed with events around
+    every replay until args.min_seconds of device time; a call's time is a
+    replay's time / REPS, so the graph's launch and the events are not charged
+    to every call.  The inputs exceed L2, so no flush is needed."""
     from fp8_kv_paged_kvq_b200 import workloads as W
     from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch
     spec = W.spec_by_name(name)
@@ -492,16 +497,17 @@ def measure_batch(name, args, dev, stream, world, e2e=True, bf16=True, cpu=True)
         for _ in range(3):
             db.step(check_tags=True, stream=stream)
         torch.cuda.synchronize()
-        g_step = capture(lambda: db.step(check_tags=True, stream=stream), stream)
-        g_nochk = capture(lambda: db.step(check_tags=False, stream=stream), stream)
-        g_dec = capture(lambda: db.decode(use_abort=True, stream=stream), stream)
+        reps = lambda f: (lambda: [f() for _ in range(REPS)])
+        g_step = capture(reps(lambda: db.step(check_tags=True, stream=stream)), stream)
+        g_nochk = capture(reps(lambda: db.step(check_tags=False, stream=stream)), stream)
+        g_dec = capture(reps(lambda: db.decode(use_abort=True, stream=stream)), stream)
         for g in (g_step, g_nochk, g_dec):
             for _ in range(3):
                 g.replay()
         barrier(world)
-        t_step = time_replays(g_step.replay, stream, args.min_seconds)
-        t_nochk = time_replays(g_nochk.replay, stream, args.min_seconds)
-        t_dec = time_replays(g_dec.replay, stream, args.min_seconds)
+        t_step = time_replays(g_step.replay, stream, args.min_seconds) / REPS
+        t_nochk = time_replays(g_nochk.replay, stream, args.min_seconds) / REPS
+        t_dec = time_replays(g_dec.replay, stream, args.min_seconds) / REPS
     st, sn, sd = stats(t_step), stats(t_nochk), stats(t_dec)
     ms_step = max_over_ranks(st["mean"], world)
     hbm, _ = peaks()
@@ -516,8 +522,9 @@ def measure_batch(name, args, dev, stream, world, e2e=True, bf16=True, cpu=True)
            "roofline": decode_roofline(s, lens, max_over_ranks(sd["mean"], world),
                                        None if is_wide(s) else
                                        measured_traffic("gqa_decode_kernel", gqa_units(s, lens))),
-           "timing": "CUDA graph replays, events around every replay, "
-                     f">= {args.min_seconds} s each; inputs exceed L2"}
+           "timing": f"CUDA graphs of {REPS} back-to-back calls, events around every "
+                     f"replay, >= {args.min_seconds} s each, per call = replay / {REPS}; "
+                     "min/median/p95 are over replays; inputs exceed L2"}
     assert_no_device_error()
     if e2e:
         res["e2e"] = run_e2e(db, args, stream, kv_bytes, world)
@@ -578,14 +585,14 @@ def run_bf16(wl_fp8, args, stream, world, dev):
     with torch.cuda.stream(stream):
         for _ in range(3):
             db.step(check_tags=True, stream=stream)
-        g = capture(lambda: db.step(check_tags=True, stream=stream), stream)
-        gd = capture(lambda: db.decode(use_abort=True, stream=stream), stream)
+        g = capture(lambda: [db.step(check_tags=True, stream=stream) for _ in range(REPS)], stream)
+        gd = capture(lambda: [db.decode(use_abort=True, stream=stream) for _ in range(REPS)], stream)
         for _ in range(3):
             g.replay()
             gd.replay()
         barrier(world)
-        t = stats(time_replays(g.replay, stream, args.min_seconds))
-        td = stats(time_replays(gd.replay, stream, args.min_seconds))
+        t = stats(time_replays(g.replay, stream, args.min_seconds) / REPS)
+        td = stats(time_replays(gd.replay, stream, args.min_seconds) / REPS)
     ms = max_over_ranks(t["mean"], world)
     msd = max_over_ranks(td["mean"], world)
     kv = 2 * wl_fp8.kv_bytes_read()
@@ -836,7 +843,8 @@ def run_ours(args):
                            "timing": res["timing"],
                            "parallelism": "replicas" if world > 1 else "single GPU"}}
         line.update({k: v for k, v in res.items() if k not in ("workload", "kv_gbs")})
-        line["gpu_launches"] = (2 + (3 if is_wide(W.spec_by_name(args.workload)) else 2)) * st["n"]
+        line["gpu_launches"] = ((2 + (3 if is_wide(W.spec_by_name(args.workload)) else 2))
+                                * st["n"] * REPS)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=8.0)
         extra = []
@@ -886,8 +894,9 @@ def run_sweep(args):
             with torch.cuda.stream(stream):
                 for _ in range(3):
                     db.decode(use_abort=False, stream=stream)
-                gd = capture(lambda: db.decode(use_abort=False, stream=stream), stream)
-                t = stats(time_replays(gd.replay, stream, args.min_seconds))
+                gd = capture(lambda: [db.decode(use_abort=False, stream=stream)
+                                      for _ in range(REPS)], stream)
+                t = stats(time_replays(gd.replay, stream, args.min_seconds) / REPS)
             kv = wl.kv_bytes_read()               # bytes of this cache format
             row[dt] = {"ms": t, "kv_gbs": kv / (t["mean"] * 1e-3) / 1e9,
                        "frac_of_hbm": kv / (t["mean"] * 1e-3) / 1e9 / hbm,

@@ -144,6 +144,18 @@ __device__ void block_prefix_units(const GqaParams& p, int32_t* pre, int32_t* sc
   __syncthreads();
 }
 
+// CTAs (or CTA pairs) that get units: at most num_ctas, at least min_units
+// units each when there are enough (the 8-head kernel asks for
+// kMinTilesPerCta: fewer, longer ranges for small batches, so fewer pieces to
+// merge and more tiles in flight per warp), and never more than U, so that
+// every working CTA owns at least one unit.  A decode kernel and the combine
+// that merges its partials use the same min_units.
+constexpr int32_t kMinTilesPerCta = 32;
+__device__ __forceinline__ int64_t working_ctas(int64_t num_ctas, int64_t U, int64_t min_units) {
+  const int64_t n = U / min_units;
+  return min(num_ctas, n > 1 ? n : (U > 0 ? int64_t{1} : int64_t{0}));
+}
+
 // Segment containing unit u: largest b with pre[b] <= u (pre has B+1 entries).
 __device__ __forceinline__ int find_seq(const int32_t* pre, int B, int32_t u) {
   int lo = 0, hi = B;            // invariant: pre[lo] <= u < pre[hi]
@@ -235,15 +247,15 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
   // and writes nothing to global memory: it lays out the units as if no
   // request were aborted and looks up its first pages.  After the wait it
   // reads the abort mask and redoes the plan only if some request aborted.
-  // The units go to the first N = min(num_ctas, U) CTAs, so that every
-  // working CTA has at least one (the combine relies on it).
+  // The units go to the first N = working_ctas(num_ctas, U) CTAs, every one
+  // of which owns at least one unit (the combine relies on it).
   const int cw = warp;
   int64_t U = 0, N = 0;
   int32_t u0 = 0, u1 = 0, kw = 0;
   auto plan = [&](bool use_abort) {
     block_prefix_units(p, pre, scratch, use_abort);  // includes __syncthreads
     U = pre[p.B];
-    N = min(static_cast<int64_t>(p.num_ctas), U);
+    N = working_ctas(p.num_ctas, U, kMinTilesPerCta);
     const bool works = static_cast<int64_t>(blockIdx.x) < N;
     u0 = works ? static_cast<int32_t>(U * blockIdx.x / N) : 0;
     u1 = works ? static_cast<int32_t>(U * (blockIdx.x + 1) / N) : 0;
@@ -624,7 +636,7 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
 // ---------------------------------------------------------------------------
 // Log-sum-exp combine.  Grid (segment = (sequence, KV head), head chunk): a
 // block merges the partials of up to kCombHeads query heads of one segment.
-// The decode launch gave its units to N = min(num_ctas, U) CTAs, CTA c taking
+// The decode launch gave its units to N = working_ctas(num_ctas, U) CTAs, CTA c taking
 // [c*U/N, (c+1)*U/N), so unit u belongs to CTA ((u+1)*N - 1) / U and the
 // pieces of a segment with units [S, E) are exactly the CTAs cs..ce that own
 // S and E - 1, every one of them non-empty.  With up to kCombFast pieces
@@ -639,13 +651,14 @@ struct CombineParams {
   const float* ws_lse;
   const float* ws_o;
   int32_t B, Hkv, G, Hq, Dv, num_ctas, heads_per_block;
+  int32_t min_units;    // the decode kernel's least units per working CTA
   float* out;
   float* lse;
 };
 
 constexpr int kCombHeads = 32;        // heads per block at most
 constexpr int kCombChunk = 64;        // pieces whose weights are staged at once
-constexpr int kCombOutputs = 4096;    // outputs per block (heads_per_block * Dv) at most
+constexpr int kCombOutputs = 2048;    // outputs per block (heads_per_block * Dv) at most
 constexpr int kCombMaxThreads = kCombOutputs / 4;   // one group of four outputs per thread
 constexpr int kCombFast = 4;          // pieces merged from registers in one round of loads
 
@@ -659,6 +672,10 @@ __device__ __forceinline__ int64_t owner_cta(int64_t u, int64_t N, int64_t U) {
 // blocks are small and all of a launch's blocks are resident at once.
 __global__ void __launch_bounds__(kCombMaxThreads) lse_combine_kernel(const CombineParams p) {
   pdl_wait();                                    // the decode kernel has finished
+  // Only now may a kernel launched after this one start (its work before its
+  // own wait then overlaps the merge): a tag check writes its clean result
+  // before its wait, and the decode kernel reads the abort mask until it ends.
+  pdl_trigger();
   const int32_t seg = blockIdx.x;
   const int32_t b = seg / p.Hkv, h = seg - b * p.Hkv;
   const int32_t h0 = blockIdx.y * p.heads_per_block;            // first head of this block
@@ -691,7 +708,7 @@ __global__ void __launch_bounds__(kCombMaxThreads) lse_combine_kernel(const Comb
   }
   // U >= tiles_b > 0 here
   const int64_t S = p.ws_pre[b] + static_cast<int64_t>(h) * tiles_b, E = S + tiles_b;
-  const int64_t N = min(static_cast<int64_t>(p.num_ctas), U);
+  const int64_t N = working_ctas(p.num_ctas, U, p.min_units);
   const int64_t cs = owner_cta(S, N, U);
   const int np = static_cast<int>(owner_cta(E - 1, N, U) - cs + 1);
   const int64_t slot0 = cs + seg;               // slot of piece k: slot0 + k
@@ -797,8 +814,10 @@ __global__ void __launch_bounds__(kCombMaxThreads) lse_combine_kernel(const Comb
 // ---------------------------------------------------------------------------
 cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const float* ws_o,
                                int32_t B, int32_t Hkv, int32_t G, int32_t Hq, int32_t Dv,
-                               int32_t num_ctas, float* out, float* lse, cudaStream_t stream) {
+                               int32_t num_ctas, int32_t min_units, float* out, float* lse,
+                               cudaStream_t stream) {
   CombineParams cp;
+  cp.min_units = min_units < 1 ? 1 : min_units;
   cp.ws_pre = ws_pre;
   cp.ws_lse = ws_lse;
   cp.ws_o = ws_o;
@@ -871,7 +890,7 @@ static cudaError_t run_gqa(const DecodeArgs& a, const CUtensorMap& km, const CUt
   e = launch_pdl(kern, dim3(a.num_ctas), dim3(K::kThreads), smem, a.stream, km, vm, p);
   if (e != cudaSuccess) return e;
   return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, a.c.Hkv, p.G, a.Hq, a.c.Dv,
-                            a.num_ctas, a.out, a.lse, a.stream);
+                            a.num_ctas, kMinTilesPerCta, a.out, a.lse, a.stream);
 }
 
 // Consumer warps and pipeline depth per configuration.

@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // working pair has at least one (the combine relies on it); the others
   // get an empty range and only set up and tear down.
   const int64_t U = __ldg(p.ws_pre + p.B);
-  const int64_t N = min(static_cast<int64_t>(p.num_pairs), U);
+  const int64_t N = working_ctas(p.num_pairs, U, 1);     // min(pairs, U)
   const bool works = pair < N;
   const int32_t u0 = works ? static_cast<int32_t>(U * pair / N) : 0;
   const int32_t u1 = works ? static_cast<int32_t>(U * (pair + 1) / N) : 0;
@@ -899,7 +899,7 @@ cudaError_t launch_wide_decode(const DecodeArgs& a, const CUtensorMap& kqk,
   e = cudaLaunchKernelEx(&cfg, wide::wide_decode_kernel, kqk, ktail, p);
   if (e != cudaSuccess) return e;
   return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, 1, wide::kHq, wide::kHq, wide::kDv,
-                            a.num_ctas, a.out, a.lse, a.stream);
+                            a.num_ctas, 1, a.out, a.lse, a.stream);
 }
 
 }  // namespace kvq

@@ -230,7 +230,10 @@ size_t kvq_decode_workspace_size(const kvq_cache* cache, int32_t B, int32_t num_
  * its split while that work may still run (the kernel launched just before
  * must not write them; kvq_validate and kvq_append never do) and everything
  * else, the abort mask included, after it has finished; the wide kernels
- * wait before reading any argument.
+ * wait before reading any argument.  The last kernel of the call (the
+ * log-sum-exp combine) lets the next kernel on the stream start once the
+ * decode kernel has finished, while it still writes out and lse: a kernel
+ * that follows must wait for its predecessor before reading them.
  */
 kvq_status kvq_decode(const kvq_cache* cache, const void* q, int32_t num_q_heads,
                       const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens,

@@ -499,10 +499,11 @@ def test_append_every_bf16_pattern(mode):
 
 @pytest.mark.parametrize("num_ctas", [0, 1000])
 def test_single_long_sequence_split_into_many_pieces(num_ctas):
-    """One sequence on one KV head: every 16-token tile can become its own
-    piece (256 pieces at 4,096 tokens with the default CTA count), so the
-    combine merges far more than one warp's worth of partials per head."""
-    spec = W.Spec("one_long", [4096], 16, 8, 1, 128, 128, outlier_p=0.01)
+    """One 40,000-token sequence on one KV head: its 2,500 tiles go to 78
+    CTAs of at least 32 tiles, so the one segment has 78 pieces and the
+    combine merges them in two chunks, far more than one warp's worth of
+    partials per head."""
+    spec = W.Spec("one_long", [40000], 16, 8, 1, 128, 128, outlier_p=0.01)
     wl, db, oc = build_both(spec, seed=16, num_ctas=num_ctas)
     out, lse = db.step(check_tags=False)
     torch.cuda.synchronize()
