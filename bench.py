@@ -77,6 +77,8 @@ def parse(argv=None):
                     help="decode steps of the long workload's loop")
     ap.add_argument("--min-seconds", type=float, default=0.5,
                     help="least device time of each timed single-batch measurement")
+    ap.add_argument("--idle-seconds", type=float, default=3.0,
+                    help="idle time before each single-batch measurement")
     ap.add_argument("--sweep", action="store_true",
                     help="capacity and concurrency sweep (FP8 vs BF16 at B = 1..64) instead of the bench line")
     ap.add_argument("--seqs", type=int, default=0,
@@ -493,7 +495,12 @@ def measure_batch(name, args, dev, stream, world, e2e=True, bf16=True, cpu=True)
     torch.cuda.synchronize()
     kv_bytes = wl.kv_bytes_read()
     s = spec
-    with torch.cuda.stream(stream):
+    # start from an idle GPU: a batch measured right after the long loop's
+    # seconds under the power cap would inherit that power state
+    torch.cuda.synchronize()
+    time.sleep(args.idle_seconds)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    with torch.cuda.stream(stream), sampler:
         for _ in range(3):
             db.step(check_tags=True, stream=stream)
         torch.cuda.synchronize()
@@ -524,7 +531,9 @@ def measure_batch(name, args, dev, stream, world, e2e=True, bf16=True, cpu=True)
                                        measured_traffic("gqa_decode_kernel", gqa_units(s, lens))),
            "timing": f"CUDA graphs of {REPS} back-to-back calls, events around every "
                      f"replay, >= {args.min_seconds} s each, per call = replay / {REPS}; "
-                     "min/median/p95 are over replays; inputs exceed L2"}
+                     "min/median/p95 are over replays; inputs exceed L2; "
+                     f"after {args.idle_seconds} s idle",
+           "clocks": sampler.summary()}
     assert_no_device_error()
     if e2e:
         res["e2e"] = run_e2e(db, args, stream, kv_bytes, world)
