@@ -118,6 +118,19 @@ def gqa_units(spec, seq_lens):
     return int(((lens + 15) // 16).sum()) * spec.num_kv_heads
 
 
+def wide_units(seq_lens):
+    """Work units of the tensor-core kernel: 64-token blocks per sequence."""
+    lens = np.asarray(seq_lens, np.int64)
+    return int(((lens + 63) // 64).sum())
+
+
+def decode_traffic(spec, seq_lens):
+    """Recorded DRAM bytes of the launch that decodes these rows, or None."""
+    if is_wide(spec):
+        return measured_traffic("wide_decode_kernel", wide_units(seq_lens))
+    return measured_traffic("gqa_decode_kernel", gqa_units(spec, seq_lens))
+
+
 def _peaks_file():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -527,8 +540,7 @@ def measure_batch(name, args, dev, stream, world, e2e=True, bf16=True, cpu=True)
            "ms_per_step": st, "ms_per_step_without_validation": sn, "ms_decode_call": sd,
            "validate_overhead_pct": 100.0 * (st["mean"] - sn["mean"]) / sn["mean"],
            "roofline": decode_roofline(s, lens, max_over_ranks(sd["mean"], world),
-                                       None if is_wide(s) else
-                                       measured_traffic("gqa_decode_kernel", gqa_units(s, lens))),
+                                       decode_traffic(s, lens)),
            "timing": f"CUDA graphs of {REPS} back-to-back calls, events around every "
                      f"replay, >= {args.min_seconds} s each, per call = replay / {REPS}; "
                      "min/median/p95 are over replays; inputs exceed L2; "

@@ -99,7 +99,7 @@ struct GqaParams {
   float sm_scale;
   float* out;
   float* lse;
-  int32_t* ws_pre;   // [B+1] unit prefix (written by CTA 0)
+  int32_t* ws_pre;   // [B+2] unit prefix, then the count of working CTAs (written by CTA 0)
   float* ws_lse;     // [slots][G]
   float* ws_o;       // [slots][G][Dv]
   int32_t num_ctas;
@@ -148,8 +148,8 @@ __device__ void block_prefix_units(const GqaParams& p, int32_t* pre, int32_t* sc
 // units each when there are enough (the 8-head kernel asks for
 // kMinTilesPerCta: fewer, longer ranges for small batches, so fewer pieces to
 // merge and more tiles in flight per warp), and never more than U, so that
-// every working CTA owns at least one unit.  A decode kernel and the combine
-// that merges its partials use the same min_units.
+// every working CTA owns at least one unit.  The decode kernels write the
+// count they used next to the unit prefix, where the combine reads it.
 constexpr int32_t kMinTilesPerCta = 32;
 __device__ __forceinline__ int64_t working_ctas(int64_t num_ctas, int64_t U, int64_t min_units) {
   const int64_t n = U / min_units;
@@ -247,15 +247,33 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
   // and writes nothing to global memory: it lays out the units as if no
   // request were aborted and looks up its first pages.  After the wait it
   // reads the abort mask and redoes the plan only if some request aborted.
-  // The units go to the first N = working_ctas(num_ctas, U) CTAs, every one
-  // of which owns at least one unit (the combine relies on it).
+  // The units go to the first N CTAs, every one of which owns at least one
+  // unit (the combine relies on it).
   const int cw = warp;
   int64_t U = 0, N = 0;
   int32_t u0 = 0, u1 = 0, kw = 0;
   auto plan = [&](bool use_abort) {
     block_prefix_units(p, pre, scratch, use_abort);  // includes __syncthreads
     U = pre[p.B];
-    N = working_ctas(p.num_ctas, U, kMinTilesPerCta);
+    // Every sequence as long as the others (in tiles) and at least two CTAs
+    // per segment: each segment gets the same number k >= 1 of CTAs, so CTA
+    // boundaries fall on segment boundaries and no CTA holds two pieces.
+    // Otherwise (ragged batches, or one CTA per segment at most, where the
+    // idle CTAs would cost more than the extra pieces) the stream-K split.
+    const int32_t t0 = p.B > 0 ? pre[1] - pre[0] : 0;
+    int uneven = 0;
+    for (int b = threadIdx.x; b < p.B; b += blockDim.x) uneven |= (pre[b + 1] - pre[b]) != t0;
+    uneven = __syncthreads_or(uneven);
+    const int64_t segs = static_cast<int64_t>(p.B) * p.c.Hkv;
+    if (!uneven && t0 > 0 && 2 * segs <= p.num_ctas) {
+      const int64_t tseg = U / segs;               // tiles of one segment
+      int64_t k = p.num_ctas / segs;
+      const int64_t kmax = tseg / kMinTilesPerCta;
+      k = min(k, kmax > 1 ? kmax : int64_t{1});
+      N = segs * k;
+    } else {
+      N = working_ctas(p.num_ctas, U, kMinTilesPerCta);
+    }
     const bool works = static_cast<int64_t>(blockIdx.x) < N;
     u0 = works ? static_cast<int32_t>(U * blockIdx.x / N) : 0;
     u1 = works ? static_cast<int32_t>(U * (blockIdx.x + 1) / N) : 0;
@@ -294,8 +312,10 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
       lookup(32, nxt_page, nxt_hy);
     }
   }
-  if (blockIdx.x == 0)
+  if (blockIdx.x == 0) {
     for (int b = threadIdx.x; b <= p.B; b += blockDim.x) p.ws_pre[b] = pre[b];
+    if (threadIdx.x == 0) p.ws_pre[p.B + 1] = static_cast<int32_t>(N);
+  }
   if (u0 >= u1) return;                          // no units: nothing issued, nothing to wait on
 
   // ---------------- this warp's pipeline ----------------
@@ -636,31 +656,28 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
 // ---------------------------------------------------------------------------
 // Log-sum-exp combine.  Grid (segment = (sequence, KV head), head chunk): a
 // block merges the partials of up to kCombHeads query heads of one segment.
-// The decode launch gave its units to N = working_ctas(num_ctas, U) CTAs, CTA c taking
+// The decode launch gave its units to N CTAs (the count it wrote after the
+// unit prefix), CTA c taking
 // [c*U/N, (c+1)*U/N), so unit u belongs to CTA ((u+1)*N - 1) / U and the
 // pieces of a segment with units [S, E) are exactly the CTAs cs..ce that own
-// S and E - 1, every one of them non-empty.  With up to kCombFast pieces
-// each thread loads its four outputs' partials from every piece in one round
-// and merges them itself: out = sum_k exp(lse_k - M) / L * o_k with M the
-// largest lse_k and L the sum of exp(lse_k - M).  With more pieces, warp w
-// first forms M and L for its heads, and the block then takes the pieces in
-// chunks of kCombChunk whose weights it stages in shared memory.
+// S and E - 1, every one of them non-empty.  Each thread merges the pieces
+// of its four outputs itself: out = sum_k exp(lse_k - M) / L * o_k with M the
+// largest lse_k and L the sum of exp(lse_k - M), taking the pieces in groups
+// of kCombGroup with a running maximum and sum, any number of them.
 // ---------------------------------------------------------------------------
 struct CombineParams {
   const int32_t* ws_pre;
   const float* ws_lse;
   const float* ws_o;
-  int32_t B, Hkv, G, Hq, Dv, num_ctas, heads_per_block;
-  int32_t min_units;    // the decode kernel's least units per working CTA
+  int32_t B, Hkv, G, Hq, Dv, heads_per_block;
   float* out;
   float* lse;
 };
 
 constexpr int kCombHeads = 32;        // heads per block at most
-constexpr int kCombChunk = 64;        // pieces whose weights are staged at once
 constexpr int kCombOutputs = 2048;    // outputs per block (heads_per_block * Dv) at most
 constexpr int kCombMaxThreads = kCombOutputs / 4;   // one group of four outputs per thread
-constexpr int kCombFast = 4;          // pieces merged from registers in one round of loads
+constexpr int kCombGroup = 4;         // pieces per round of loads
 
 // CTA of a launch with N working CTAs over U units that owns unit u.
 __device__ __forceinline__ int64_t owner_cta(int64_t u, int64_t N, int64_t U) {
@@ -670,7 +687,7 @@ __device__ __forceinline__ int64_t owner_cta(int64_t u, int64_t N, int64_t U) {
 // One thread per group of four consecutive output dims of the block's heads
 // (blockDim = heads_per_block * Dv / 4, at most kCombMaxThreads), so the
 // blocks are small and all of a launch's blocks are resident at once.
-__global__ void __launch_bounds__(kCombMaxThreads) lse_combine_kernel(const CombineParams p) {
+__global__ void __launch_bounds__(kCombMaxThreads, 2) lse_combine_kernel(const CombineParams p) {
   pdl_wait();                                    // the decode kernel has finished
   // Only now may a kernel launched after this one start (its work before its
   // own wait then overlaps the merge): a tag check writes its clean result
@@ -708,105 +725,74 @@ __global__ void __launch_bounds__(kCombMaxThreads) lse_combine_kernel(const Comb
   }
   // U >= tiles_b > 0 here
   const int64_t S = p.ws_pre[b] + static_cast<int64_t>(h) * tiles_b, E = S + tiles_b;
-  const int64_t N = working_ctas(p.num_ctas, U, p.min_units);
+  const int64_t N = p.ws_pre[p.B + 1];          // the decode launch's working CTAs
   const int64_t cs = owner_cta(S, N, U);
   const int np = static_cast<int>(owner_cta(E - 1, N, U) - cs + 1);
   const int64_t slot0 = cs + seg;               // slot of piece k: slot0 + k
-  if (np <= kCombFast) {
-    // few pieces: one round of loads of this group's partial outputs and its
-    // head's partial lse from every piece, merged in registers
-    if (!mine) return;
-    float4 o[kCombFast];
-    float a[kCombFast];
+  if (!mine) return;
+  // Pieces in groups of kCombGroup with a running maximum m, sum l and
+  // output acc (rescaled by exp(m_old - m_new) when m moves); the loads of
+  // the next group are issued before the current group is merged.  A single
+  // piece comes out bit for bit (weight exp(0) = 1, l = 1).
+  const int64_t row0 = slot0 * p.G + h0 + hh;   // piece k at row0 + k * G
+  const int64_t rstep = p.G;
+  float4 o[2][kCombGroup];
+  float a[2][kCombGroup];
+  auto load_group = [&](int x, int base) {
 #pragma unroll
-    for (int k = 0; k < kCombFast; ++k) {
-      if (k < np) {
-        const int64_t row = (slot0 + k) * p.G + h0 + hh;
-        o[k] = *reinterpret_cast<const float4*>(p.ws_o + row * p.Dv + d);
-        a[k] = p.ws_lse[row];
+    for (int k = 0; k < kCombGroup; ++k) {
+      if (base + k < np) {
+        const int64_t row = row0 + static_cast<int64_t>(base + k) * rstep;
+        o[x][k] = *reinterpret_cast<const float4*>(p.ws_o + row * p.Dv + d);
+        a[x][k] = p.ws_lse[row];
       }
     }
-    float4 acc = o[0];                           // a single piece is copied bit for bit
-    float lse_h = a[0];
-    if (np > 1) {
-      float M = a[0];
-#pragma unroll
-      for (int k = 1; k < kCombFast; ++k)
-        if (k < np) M = fmaxf(M, a[k]);
-      float L = 0.0f, w[kCombFast];
-#pragma unroll
-      for (int k = 0; k < kCombFast; ++k) {
-        w[k] = k < np ? __expf(a[k] - M) : 0.0f;
-        L += w[k];
-      }
-      const float inv = 1.0f / L;
-      acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < kCombFast; ++k) {
-        if (k < np) {
-          const float wk = w[k] * inv;
-          acc.x += wk * o[k].x;
-          acc.y += wk * o[k].y;
-          acc.z += wk * o[k].z;
-          acc.w += wk * o[k].w;
-        }
-      }
-      lse_h = M + __logf(L);
-    }
-    if (lse && d == 0) lse[hh] = lse_h;
-    store(acc);
-    return;
-  }
-  // many pieces: warp w forms the maximum M and the sum L for heads w,
-  // w + warps, ...; then the block takes the pieces in chunks whose weights
-  // exp(lse_k - M) / L it stages in shared memory
-  __shared__ float m_sh[kCombHeads], inv_sh[kCombHeads];
-  __shared__ float wts[kCombHeads][kCombChunk];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
+  };
   const float kNegInf = -__int_as_float(0x7f800000);
-  for (int x = warp; x < nh; x += nwarps) {
-    const float* l = p.ws_lse + slot0 * p.G + h0 + x;   // piece k at l[k * G]
-    float M = kNegInf;
-    for (int k = lane; k < np; k += 32) M = fmaxf(M, l[static_cast<int64_t>(k) * p.G]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.0f;
-    for (int k = lane; k < np; k += 32) L += __expf(l[static_cast<int64_t>(k) * p.G] - M);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) {
-      m_sh[x] = M;
-      inv_sh[x] = 1.0f / L;
-      if (lse) lse[x] = M + __logf(L);
-    }
-  }
-  __syncthreads();                               // m_sh, inv_sh
+  float m = kNegInf, l = 0.0f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int base = 0; base < np; base += kCombChunk) {
-    const int nk = min(kCombChunk, np - base);
-    for (int idx = threadIdx.x; idx < nh * nk; idx += blockDim.x) {
-      const int x = idx / nk, k = idx - x * nk;
-      const float a = p.ws_lse[(slot0 + base + k) * p.G + h0 + x];
-      wts[x][k] = __expf(a - m_sh[x]) * inv_sh[x];
-    }
-    __syncthreads();
-    if (mine) {
-      const float* o = p.ws_o + ((slot0 + base) * p.G + h0 + hh) * p.Dv + d;
-      const int64_t stride = static_cast<int64_t>(p.G) * p.Dv;   // next piece
-#pragma unroll 4
-      for (int k = 0; k < nk; ++k) {
-        const float4 v = *reinterpret_cast<const float4*>(o + k * stride);
-        const float w = wts[hh][k];
-        acc.x += w * v.x;
-        acc.y += w * v.y;
-        acc.z += w * v.z;
-        acc.w += w * v.w;
+  auto merge = [&](int x, int base) {
+    float mg = m;
+#pragma unroll
+    for (int k = 0; k < kCombGroup; ++k)
+      if (base + k < np) mg = fmaxf(mg, a[x][k]);
+    const float r = __expf(m - mg);                // 0 on the first group
+    l *= r;
+    acc.x *= r;
+    acc.y *= r;
+    acc.z *= r;
+    acc.w *= r;
+#pragma unroll
+    for (int k = 0; k < kCombGroup; ++k) {
+      if (base + k < np) {
+        const float w = __expf(a[x][k] - mg);
+        l += w;
+        acc.x += w * o[x][k].x;
+        acc.y += w * o[x][k].y;
+        acc.z += w * o[x][k].z;
+        acc.w += w * o[x][k].w;
       }
     }
-    __syncthreads();                             // wts reused by the next chunk
+    m = mg;
+  };
+  // two buffers used alternately with constant indices (registers)
+  load_group(0, 0);
+  for (int base = 0; base < np; base += 2 * kCombGroup) {
+    if (base + kCombGroup < np) load_group(1, base + kCombGroup);
+    merge(0, base);
+    if (base + kCombGroup >= np) break;
+    if (base + 2 * kCombGroup < np) load_group(0, base + 2 * kCombGroup);
+    merge(1, base + kCombGroup);
   }
-  if (mine) store(acc);
+  if (np > 1) {
+    const float inv = 1.0f / l;
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
+  }
+  if (lse && d == 0) lse[hh] = np == 1 ? m : m + __logf(l);
+  store(acc);
 }
 
 // ---------------------------------------------------------------------------
@@ -814,10 +800,8 @@ __global__ void __launch_bounds__(kCombMaxThreads) lse_combine_kernel(const Comb
 // ---------------------------------------------------------------------------
 cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const float* ws_o,
                                int32_t B, int32_t Hkv, int32_t G, int32_t Hq, int32_t Dv,
-                               int32_t num_ctas, int32_t min_units, float* out, float* lse,
-                               cudaStream_t stream) {
+                               float* out, float* lse, cudaStream_t stream) {
   CombineParams cp;
-  cp.min_units = min_units < 1 ? 1 : min_units;
   cp.ws_pre = ws_pre;
   cp.ws_lse = ws_lse;
   cp.ws_o = ws_o;
@@ -826,7 +810,6 @@ cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const
   cp.G = G;
   cp.Hq = Hq;
   cp.Dv = Dv;
-  cp.num_ctas = num_ctas;
   cp.out = out;
   cp.lse = lse;
   if (Dv % 4 != 0 || Dv > kCombOutputs) return cudaErrorInvalidValue;
@@ -890,7 +873,7 @@ static cudaError_t run_gqa(const DecodeArgs& a, const CUtensorMap& km, const CUt
   e = launch_pdl(kern, dim3(a.num_ctas), dim3(K::kThreads), smem, a.stream, km, vm, p);
   if (e != cudaSuccess) return e;
   return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, a.c.Hkv, p.G, a.Hq, a.c.Dv,
-                            a.num_ctas, kMinTilesPerCta, a.out, a.lse, a.stream);
+                            a.out, a.lse, a.stream);
 }
 
 // Consumer warps and pipeline depth per configuration.

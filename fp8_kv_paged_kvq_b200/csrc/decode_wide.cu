@@ -153,7 +153,7 @@ struct Params {
   int32_t B;
   const uint8_t* abort_mask;
   float sm_scale;
-  int32_t* ws_pre;          // [B+1] prefix of 64-token blocks (written by the pre-pass)
+  int32_t* ws_pre;          // [B+2] prefix of 64-token blocks, then the working pairs (pre-pass)
   float* ws_lse;            // [slots][128]
   float* ws_o;              // [slots][128][512]
   uint8_t* ws_q;            // [B][2][kQImage] query images (written by the pre-pass)
@@ -200,7 +200,10 @@ __global__ void __launch_bounds__(kPrepThreads) wide_prep_kernel(const Params p)
       p.ws_pre[b] = run;
       run += (seq_tokens(p, b) + kBlk - 1) / kBlk;
     }
-    if (tid == kPrepThreads - 1) p.ws_pre[p.B] = run;   // the last run ends at B
+    if (tid == kPrepThreads - 1) {
+      p.ws_pre[p.B] = run;                               // the last run ends at B
+      p.ws_pre[p.B + 1] = min(p.num_pairs, run);         // working pairs, as the decode kernel
+    }
     return;
   }
   const int b = blockIdx.x >> 1, r = blockIdx.x & 1;
@@ -899,7 +902,7 @@ cudaError_t launch_wide_decode(const DecodeArgs& a, const CUtensorMap& kqk,
   e = cudaLaunchKernelEx(&cfg, wide::wide_decode_kernel, kqk, ktail, p);
   if (e != cudaSuccess) return e;
   return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, 1, wide::kHq, wide::kHq, wide::kDv,
-                            a.num_ctas, 1, a.out, a.lse, a.stream);
+                            a.out, a.lse, a.stream);
 }
 
 }  // namespace kvq

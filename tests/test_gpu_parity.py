@@ -512,6 +512,30 @@ def test_single_long_sequence_split_into_many_pieces(num_ctas):
     assert kvq.device_error() == 0
 
 
+@pytest.mark.parametrize("num_ctas", [0, 5, 12, 20])
+def test_equal_tile_counts_split_on_segment_edges(num_ctas):
+    """Sequences of one tile count (126 tiles of 16 tokens each, ragged last
+    tiles), 8 segments: with at least two CTAs per segment each segment gets
+    its own CTAs (3 each by default, 2 at 20 CTAs); with 5 or 12 CTAs the
+    split falls back to the stream-K ranges.  With a stale tag one row aborts
+    and the plan redone after the wait is the stream-K one."""
+    spec = W.Spec("even_tiles", [2001, 2002, 2016, 2010], 16, 16, 2, 128, 128,
+                  outlier_p=0.01, n_stale=1)
+    wl, db, oc = build_both(spec, seed=18, num_ctas=num_ctas)
+    out, lse = db.step(check_tags=True)
+    torch.cuda.synchronize()
+    mask = db.abort.cpu().numpy()
+    ref_mask = oracle.validate(oc.page_tags, wl.block_table, wl.expected_tags, wl.seq_lens,
+                               wl.spec.page_size)
+    assert np.array_equal(mask, ref_mask) and mask.sum() == 1
+    ro, rl = OS.decode(wl, oc, abort=ref_mask)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), "aborted")
+    out2, lse2 = db.decode(use_abort=False)
+    ro2, rl2 = OS.decode(wl, oc, abort=None)
+    assert_decode_close(out2, lse2, ro2.reshape(out.shape), rl2.reshape(lse.shape), "even")
+    assert kvq.device_error() == 0
+
+
 def test_few_kv_heads_long_context_bf16_and_group_16():
     """B = 1 with four KV heads (about 74 pieces per segment at the default
     CTA count) on the BF16 cache, and a 16-head group on the FP8 cache."""
