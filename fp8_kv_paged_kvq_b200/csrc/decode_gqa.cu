@@ -660,34 +660,39 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
 // unit prefix), CTA c taking
 // [c*U/N, (c+1)*U/N), so unit u belongs to CTA ((u+1)*N - 1) / U and the
 // pieces of a segment with units [S, E) are exactly the CTAs cs..ce that own
-// S and E - 1, every one of them non-empty.  Each thread merges the pieces
-// of its four outputs itself: out = sum_k exp(lse_k - M) / L * o_k with M the
-// largest lse_k and L the sum of exp(lse_k - M), taking the pieces in groups
-// of kCombGroup with a running maximum and sum, any number of them.
+// S and E - 1, every one of them non-empty.  out = sum_k exp(lse_k - M) / L *
+// o_k with M the largest lse_k and L the sum of exp(lse_k - M).  Each group
+// of four outputs has 2^lanes_log2 consecutive threads (sub-lanes): sub-lane
+// j takes pieces j, j + 2^lanes_log2, ... in rounds of kCombGroup loads with
+// a running maximum and sum, any number of them, and the sub-lanes' states
+// are then merged pairwise through shuffles.  Several sub-lanes serve
+// segments split into many pieces (small batches), where one thread's rounds
+// of loads would follow one another.
 // ---------------------------------------------------------------------------
 struct CombineParams {
   const int32_t* ws_pre;
   const float* ws_lse;
   const float* ws_o;
-  int32_t B, Hkv, G, Hq, Dv, heads_per_block;
+  int32_t B, Hkv, G, Hq, Dv, heads_per_block, lanes_log2;
   float* out;
   float* lse;
 };
 
 constexpr int kCombHeads = 32;        // heads per block at most
 constexpr int kCombOutputs = 2048;    // outputs per block (heads_per_block * Dv) at most
-constexpr int kCombMaxThreads = kCombOutputs / 4;   // one group of four outputs per thread
+constexpr int kCombMaxThreads = kCombOutputs / 4;   // threads per block at most
 constexpr int kCombGroup = 4;         // pieces per round of loads
+constexpr int kCombMaxLanesLog2 = 3;  // at most 8 sub-lanes per group of four outputs
 
 // CTA of a launch with N working CTAs over U units that owns unit u.
 __device__ __forceinline__ int64_t owner_cta(int64_t u, int64_t N, int64_t U) {
   return ((u + 1) * N - 1) / U;
 }
 
-// One thread per group of four consecutive output dims of the block's heads
-// (blockDim = heads_per_block * Dv / 4, at most kCombMaxThreads), so the
-// blocks are small and all of a launch's blocks are resident at once.
-__global__ void __launch_bounds__(kCombMaxThreads, 2) lse_combine_kernel(const CombineParams p) {
+// blockDim = heads_per_block * Dv / 4 * 2^lanes_log2 (in whole warps, at
+// most kCombMaxThreads), so the blocks are small.  No minimum of resident
+// blocks is asked for: under 64 registers the double-buffered loads spill.
+__global__ void __launch_bounds__(kCombMaxThreads, 1) lse_combine_kernel(const CombineParams p) {
   pdl_wait();                                    // the decode kernel has finished
   // Only now may a kernel launched after this one start (its work before its
   // own wait then overlaps the merge): a tag check writes its clean result
@@ -703,7 +708,9 @@ __global__ void __launch_bounds__(kCombMaxThreads, 2) lse_combine_kernel(const C
   float* lse = p.lse ? p.lse + static_cast<int64_t>(b) * p.Hq + h * p.G + h0 : nullptr;
   const int dq = p.Dv >> 2;                     // outputs in groups of four dims
   const int n4 = nh * dq;
-  const int i4 = threadIdx.x;                   // this thread's group
+  const int lg = p.lanes_log2, nl = 1 << lg;
+  const int i4 = threadIdx.x >> lg;             // this thread's group
+  const int sub = threadIdx.x & (nl - 1);       // and its sub-lane in the group
   const bool mine = i4 < n4;
   const int hh = mine ? i4 / dq : 0, d = mine ? (i4 - hh * dq) * 4 : 0;
   const bool vec_out = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
@@ -718,9 +725,9 @@ __global__ void __launch_bounds__(kCombMaxThreads, 2) lse_combine_kernel(const C
       dst[3] = acc.w;
     }
   };
-  if (tiles_b == 0) {
-    if (mine) store(make_float4(0.f, 0.f, 0.f, 0.f));
-    if (lse && mine && d == 0) lse[hh] = -__int_as_float(0x7f800000);
+  if (tiles_b == 0) {                           // the same for the whole block
+    if (mine && sub == 0) store(make_float4(0.f, 0.f, 0.f, 0.f));
+    if (lse && mine && sub == 0 && d == 0) lse[hh] = -__int_as_float(0x7f800000);
     return;
   }
   // U >= tiles_b > 0 here
@@ -729,19 +736,21 @@ __global__ void __launch_bounds__(kCombMaxThreads, 2) lse_combine_kernel(const C
   const int64_t cs = owner_cta(S, N, U);
   const int np = static_cast<int>(owner_cta(E - 1, N, U) - cs + 1);
   const int64_t slot0 = cs + seg;               // slot of piece k: slot0 + k
-  if (!mine) return;
-  // Pieces in groups of kCombGroup with a running maximum m, sum l and
-  // output acc (rescaled by exp(m_old - m_new) when m moves); the loads of
-  // the next group are issued before the current group is merged.  A single
-  // piece comes out bit for bit (weight exp(0) = 1, l = 1).
-  const int64_t row0 = slot0 * p.G + h0 + hh;   // piece k at row0 + k * G
-  const int64_t rstep = p.G;
+  // This sub-lane's pieces sub, sub + nl, ... (none for threads past the
+  // block's outputs, which still take part in the shuffles), in groups of
+  // kCombGroup with a running maximum m, sum l and output acc (rescaled by
+  // exp(m_old - m_new) when m moves); the loads of the next group are issued
+  // before the current group is merged.  A single piece comes out bit for
+  // bit (weight exp(0) = 1, l = 1, and the empty sub-lanes weigh 0).
+  const int my_np = mine && sub < np ? (np - 1 - sub) / nl + 1 : 0;
+  const int64_t row0 = (slot0 + sub) * p.G + h0 + hh;   // my piece k at row0 + k * rstep
+  const int64_t rstep = static_cast<int64_t>(nl) * p.G;
   float4 o[2][kCombGroup];
   float a[2][kCombGroup];
   auto load_group = [&](int x, int base) {
 #pragma unroll
     for (int k = 0; k < kCombGroup; ++k) {
-      if (base + k < np) {
+      if (base + k < my_np) {
         const int64_t row = row0 + static_cast<int64_t>(base + k) * rstep;
         o[x][k] = *reinterpret_cast<const float4*>(p.ws_o + row * p.Dv + d);
         a[x][k] = p.ws_lse[row];
@@ -755,7 +764,7 @@ __global__ void __launch_bounds__(kCombMaxThreads, 2) lse_combine_kernel(const C
     float mg = m;
 #pragma unroll
     for (int k = 0; k < kCombGroup; ++k)
-      if (base + k < np) mg = fmaxf(mg, a[x][k]);
+      if (base + k < my_np) mg = fmaxf(mg, a[x][k]);
     const float r = __expf(m - mg);                // 0 on the first group
     l *= r;
     acc.x *= r;
@@ -764,7 +773,7 @@ __global__ void __launch_bounds__(kCombMaxThreads, 2) lse_combine_kernel(const C
     acc.w *= r;
 #pragma unroll
     for (int k = 0; k < kCombGroup; ++k) {
-      if (base + k < np) {
+      if (base + k < my_np) {
         const float w = __expf(a[x][k] - mg);
         l += w;
         acc.x += w * o[x][k].x;
@@ -777,13 +786,33 @@ __global__ void __launch_bounds__(kCombMaxThreads, 2) lse_combine_kernel(const C
   };
   // two buffers used alternately with constant indices (registers)
   load_group(0, 0);
-  for (int base = 0; base < np; base += 2 * kCombGroup) {
-    if (base + kCombGroup < np) load_group(1, base + kCombGroup);
+  for (int base = 0; base < my_np; base += 2 * kCombGroup) {
+    if (base + kCombGroup < my_np) load_group(1, base + kCombGroup);
     merge(0, base);
-    if (base + kCombGroup >= np) break;
-    if (base + 2 * kCombGroup < np) load_group(0, base + 2 * kCombGroup);
+    if (base + kCombGroup >= my_np) break;
+    if (base + 2 * kCombGroup < my_np) load_group(0, base + 2 * kCombGroup);
     merge(1, base + kCombGroup);
   }
+  // merge the sub-lanes' states pairwise (an empty state has m = -inf, l = 0)
+  for (int x = 1; x < nl; x <<= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, x);
+    const float l2 = __shfl_xor_sync(0xffffffffu, l, x);
+    float4 a2;
+    a2.x = __shfl_xor_sync(0xffffffffu, acc.x, x);
+    a2.y = __shfl_xor_sync(0xffffffffu, acc.y, x);
+    a2.z = __shfl_xor_sync(0xffffffffu, acc.z, x);
+    a2.w = __shfl_xor_sync(0xffffffffu, acc.w, x);
+    const float mg = fmaxf(m, m2);
+    const float ref = mg == -__int_as_float(0x7f800000) ? 0.0f : mg;
+    const float f1 = __expf(m - ref), f2 = __expf(m2 - ref);
+    l = l * f1 + l2 * f2;
+    acc.x = acc.x * f1 + a2.x * f2;
+    acc.y = acc.y * f1 + a2.y * f2;
+    acc.z = acc.z * f1 + a2.z * f2;
+    acc.w = acc.w * f1 + a2.w * f2;
+    m = mg;
+  }
+  if (!mine || sub != 0) return;
   if (np > 1) {
     const float inv = 1.0f / l;
     acc.x *= inv;
@@ -800,7 +829,7 @@ __global__ void __launch_bounds__(kCombMaxThreads, 2) lse_combine_kernel(const C
 // ---------------------------------------------------------------------------
 cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const float* ws_o,
                                int32_t B, int32_t Hkv, int32_t G, int32_t Hq, int32_t Dv,
-                               float* out, float* lse, cudaStream_t stream) {
+                               int32_t num_ctas, float* out, float* lse, cudaStream_t stream) {
   CombineParams cp;
   cp.ws_pre = ws_pre;
   cp.ws_lse = ws_lse;
@@ -813,12 +842,23 @@ cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const
   cp.out = out;
   cp.lse = lse;
   if (Dv % 4 != 0 || Dv > kCombOutputs) return cudaErrorInvalidValue;
-  int hpb = kCombOutputs / Dv;
+  // Sub-lanes: a segment has about num_ctas / segments + 1 pieces.  Up to
+  // two rounds of loads stay on one thread; beyond that each sub-lane gets
+  // up to kCombGroup pieces (one round), with at most 2^kCombMaxLanesLog2
+  // sub-lanes and one head's groups within a block.
+  const int64_t segs = static_cast<int64_t>(B) * Hkv;
+  const int64_t pieces = (segs > 0 ? num_ctas / segs : 0) + 1;
+  int lg = 0;
+  if (pieces > 2 * kCombGroup)
+    while (lg < kCombMaxLanesLog2 && (static_cast<int64_t>(kCombGroup) << lg) < pieces) ++lg;
+  while (lg > 0 && ((Dv / 4) << lg) > kCombMaxThreads) --lg;
+  cp.lanes_log2 = lg;
+  int hpb = (kCombOutputs >> lg) / Dv;
   hpb = hpb < 1 ? 1 : (hpb > kCombHeads ? kCombHeads : hpb);
   hpb = hpb > G ? G : hpb;
   cp.heads_per_block = hpb;
-  // one thread per four outputs of the block, in whole warps
-  const int threads = (hpb * (Dv / 4) + 31) / 32 * 32;
+  // 2^lg threads per four outputs of the block, in whole warps
+  const int threads = (((hpb * (Dv / 4)) << lg) + 31) / 32 * 32;
   const dim3 grid(static_cast<unsigned>(B * Hkv), static_cast<unsigned>((G + hpb - 1) / hpb));
   if (B * Hkv == 0) return cudaSuccess;
   return launch_pdl(lse_combine_kernel, grid, dim3(threads), 0, stream, cp);
@@ -873,7 +913,7 @@ static cudaError_t run_gqa(const DecodeArgs& a, const CUtensorMap& km, const CUt
   e = launch_pdl(kern, dim3(a.num_ctas), dim3(K::kThreads), smem, a.stream, km, vm, p);
   if (e != cudaSuccess) return e;
   return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, a.c.Hkv, p.G, a.Hq, a.c.Dv,
-                            a.out, a.lse, a.stream);
+                            a.num_ctas, a.out, a.lse, a.stream);
 }
 
 // Consumer warps and pipeline depth per configuration.

@@ -75,7 +75,7 @@ size_t wide_q_image_bytes();   // per sequence, in the workspace's extra region
 cudaError_t launch_wide_decode(const DecodeArgs& a, const CUtensorMap& kqk, const CUtensorMap& ktail);
 cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const float* ws_o,
                                int32_t B, int32_t Hkv, int32_t G, int32_t Hq, int32_t Dv,
-                               float* out, float* lse, cudaStream_t stream);
+                               int32_t num_ctas, float* out, float* lse, cudaStream_t stream);
 void gqa_tma_box(bool fp8, int D, int* box_elems, int* swizzle_bytes);
 cudaError_t launch_gqa_decode(const DecodeArgs& a, const CUtensorMap& km, const CUtensorMap& vm);
 

@@ -536,6 +536,26 @@ def test_equal_tile_counts_split_on_segment_edges(num_ctas):
     assert kvq.device_error() == 0
 
 
+def test_many_short_segments_group_1():
+    """32 KV heads with one query head each and 520 short ragged rows (1..60
+    tokens, head dim 64): 16,640 segments, each CTA's range crossing about
+    fifty of them; two stale tags."""
+    B = 520
+    r = np.random.default_rng(20)
+    lens = [int(x) for x in r.integers(1, 61, B)]
+    spec = W.Spec(f"segs_{B}", lens, 16, 32, 32, 64, 64, n_stale=2)
+    wl, db, oc = build_both(spec, seed=20)
+    out, lse = db.step(check_tags=True)
+    torch.cuda.synchronize()
+    mask = db.abort.cpu().numpy()
+    ref_mask = oracle.validate(oc.page_tags, wl.block_table, wl.expected_tags, wl.seq_lens,
+                               wl.spec.page_size)
+    assert np.array_equal(mask, ref_mask)
+    ro, rl = OS.decode(wl, oc, abort=ref_mask)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), spec.name)
+    assert kvq.device_error() == 0
+
+
 def test_few_kv_heads_long_context_bf16_and_group_16():
     """B = 1 with four KV heads (about 74 pieces per segment at the default
     CTA count) on the BF16 cache, and a 16-head group on the FP8 cache."""
