@@ -31,28 +31,32 @@
 //    then PV of the block two back for value-dim half k (N = 256).  The
 //    softmax adds the partial scores; the fixed order per stream keeps PV,
 //    which frees the P and V buffers, from queuing behind QK^T.
-//  * PV: kind::f16.  P goes to f16 with the token's scale folded in; V is
-//    converted from E4M3 to f16 exactly, as V * 2^-8, by moving bits on the
-//    integer pipes (the conversion unit is left to exp2 and the P packing);
-//    the epilogue multiplies by 2^8.  Each SM converts only the 256 value
-//    dims that its halves of the two PV instructions' B operands hold.
+//  * PV: kind::f8f6f4 as well, on the stored value codes.  P, with the
+//    token's scale folded in and a per-head power of two 2^f, is split into
+//    three E4M3 terms (t0 = E4M3(v), t1 = E4M3(v - t0), t2 = E4M3(v - t0 -
+//    t1): about 12 significant bits, against the 8 of two terms, which
+//    peaky score rows showed to be too few); the power of two moves only
+//    when a block would exceed the E4M3 range (O is then rescaled in TMEM
+//    with the reference max), and the epilogue multiplies by 2^-f.
 //  * The B operand of QK^T is split by tokens between the two SMs (the
 //    leader holds tokens 0-31 of the block, the other SM tokens 32-63), and
 //    both SMs' key loads complete on the leader's barrier.  The B operand of
-//    PV is split by value dims, so the V conversion reads the 32 tokens it
-//    lacks from the other SM's stage through distributed shared memory
-//    instead of loading them again.
+//    PV is split by value dims, and a pair MMA reads both SMs' halves at the
+//    same shared-memory offset, so PV cannot read the key stage in place:
+//    each SM copies the raw code atoms of its 32 tokens (4 KB each, 128-byte
+//    swizzle kept) into its own value buffer and into the other SM's, with
+//    bulk shared-memory copies (16 KB per block per SM, no conversion).
 //  * Softmax: eight warps per SM; each thread holds one head and 16 of the
 //    block's 64 tokens (TMEM lane quarter and column half), and the four
 //    warps holding the same 32 heads exchange partial maxima and sums
 //    through shared memory.  Scores are scaled to base 2 and exponentiated
 //    against a reference max that moves only when a score exceeds it by 2^8
 //    (then O is rescaled in TMEM).
-//  * Warp roles per CTA: 0 TMA producer (three key stages, page ids read 32
+//  * Warp roles per CTA: 0 TMA producer (five key stages, page ids read 32
 //    blocks ahead); 1-2 MMA streams (leader CTA only; warp 1 also owns the
-//    tensor memory); 3-10 softmax, P and O read-out; 11-14 V conversion.
-//    S has three buffers per MMA stream; converted V and P two each, freed
-//    by the completion of the PV that read them.
+//    tensor memory); 3-10 softmax, P and O read-out; 11 token scales for the
+//    softmax and the value copies.  S has three buffers per MMA stream; V
+//    and P two each, freed by the completion of the PV that read them.
 //  * Work split as in the 8-head kernel: the pre-pass also writes the prefix
 //    of 64-token blocks over the sequences, the blocks of all sequences are
 //    split evenly over the CTA pairs (split-KV), each pair writes one
@@ -79,18 +83,20 @@ constexpr int kNumMma = KVQ_WIDE_STREAMS;             // MMA streams (2 or 4)
 static_assert(kNumMma == 2 || kNumMma == 4, "MMA streams");
 constexpr int kWarpMma = 1;                           // warps 1 .. kNumMma
 constexpr int kWarpSoftmax = kWarpMma + kNumMma;      // 8 softmax warps
-constexpr int kWarpV = kWarpSoftmax + 8;              // 4 V warps
-constexpr int kThreads = 32 * (kWarpV + 4);
+constexpr int kWarpV = kWarpSoftmax + 8;              // scales and value copies
+constexpr int kThreads = 32 * (kWarpV + 1);
 
-constexpr int kNK = 3;                                // key stages
+constexpr int kNK = 5;                                // key stages
 constexpr int kQkAtom = 32 * 128;                     // 32 token rows x 128 dims
 constexpr int kStage = 4 * kQkAtom + 32 * 64;         // + 64-dim tail: 18,432 B
 constexpr int kQAtom = 64 * 128;                      // 64 head rows x 128 dims
 constexpr int kQPart = 4 * kQAtom + 64 * 64;          // one E4M3 term: 36,864 B
 constexpr int kQImage = 2 * kQPart + kH * 4;          // hi, lo, 2^-e per head
-constexpr int kVHalf = kBlk * 128 * 2;                // 64 tokens x 128 dims f16
+constexpr int kVHalf = kBlk * 128;                    // 64 tokens x 128 value dims, E4M3
 constexpr int kVBuf = 2 * kVHalf;                     // one CTA's 256 value dims
-constexpr int kPBuf = kH * kBlk * 2;
+constexpr int kPTerms = 3;                            // E4M3 terms of P
+constexpr int kPTerm = kH * kBlk;                     // one term: 64 heads x 64 tokens
+constexpr int kPBuf = kPTerms * kPTerm;
 constexpr int kNSc = 4;                               // scale ring entries
 constexpr int kNP = 2;                                // P buffers (freed with V: kPvDone)
 constexpr int kNS = 3;                                // S buffers per MMA stream
@@ -101,22 +107,36 @@ constexpr int kOffV = kOffK + kNK * kStage;           // 2 buffers
 constexpr int kOffP = kOffV + 2 * kVBuf;              // kNP buffers
 constexpr int kOffKSc = kOffP + kNP * kPBuf;          // token scales per key stage
 constexpr int kOffScR = kOffKSc + kNK * kBlk * 4;     // scale ring read by the softmax
-constexpr int kOffXm = kOffScR + kNSc * kBlk * 4;
+constexpr int kOffScMax = kOffScR + kNSc * kBlk * 4;  // largest scale of each ring entry
+constexpr int kOffXm = kOffScMax + kNSc * 4;
 constexpr int kOffXl = kOffXm + 2 * 256 * 4;         // xm: two blocks' partial maxima
 constexpr int kOffFlag = kOffXl + 256 * 4;            // per key stage: page in range
-constexpr int kOffSink = kOffFlag + 16;               // V warps: one word each
-constexpr int kOffBars = kOffSink + 16;
+constexpr int kOffBars = kOffFlag + 32;
 enum {
   // completed in the leader CTA
-  kKFull = 0, kSFree = 3, kQReady = 6, kPReady = 7, kVReady = 9, kOFree = 11,
+  kKFull = 0,
+  kSFree = kKFull + kNK,
+  kQReady = kSFree + kNS,
+  kPReady = kQReady + 1,
+  kVReady = kPReady + 2,
+  kOFree = kVReady + 2,
   // arrive in both CTAs (multicast commits)
-  kSFull = 12, kKFree = 15, kPvDone = 18,
+  kSFull = kOFree + 1,
+  kKFree = kSFull + kNS,
+  kPvDone = kKFree + kNK,
   // local
-  kKPeerFull = 20, kScL = 23, kScR = 26, kQFull = 30, kDrain = 31, kNumBars = 35
+  kKPeerFull = kPvDone + 2,
+  kScL = kKPeerFull + kNK,
+  kScR = kScL + kNK,
+  kQFull = kScR + kNSc,
+  kVFull = kQFull + 1,
+  kDrain = kVFull + 2,
+  kNumBars = kDrain + 4
 };
 constexpr int kOffTmem = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = 1024 + kOffTmem + 16;
 static_assert(kQImage <= kOffK, "query image overlaps the key stages");
+static_assert(kNK <= 8, "stage flags");
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 // TMEM columns: O at [0, 256) (value-dim half h of the pair at 128*h), the
@@ -125,11 +145,22 @@ static_assert(256 + 32 * kNS * kNumMma <= 512, "tensor memory");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 256;
 
-// Instruction descriptors: FP32 accumulate (bit 4), M = 128 (m_dim = 8 at
-// bit 24), N >> 3 at bit 17; QK^T E4M3 x E4M3 both K-major (N = 64 tokens);
-// PV f16 x f16 with B (the values) MN-major (bit 16), N = 256 value dims.
+// Instruction descriptors (kind::f8f6f4, E4M3 x E4M3): FP32 accumulate
+// (bit 4), M = 128 (m_dim = 8 at bit 24), N >> 3 at bit 17; QK^T both
+// K-major (N = 64 tokens); PV with B (the values) MN-major (bit 16), N = 256
+// value dims.
 constexpr uint32_t kIdescQK = (1u << 4) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
+
+// 2^f as a float, f in [-126, 127]
+__device__ __forceinline__ float pow2f(int f) { return __int_as_float((f + 127) << 23); }
+// f with v * 2^f in [128, 256) for a positive normal v, held to [-120, 120]
+// (subnormal v count as 2^-127)
+__device__ __forceinline__ int pow2_exponent(float v) {
+  const int e = static_cast<int>((__float_as_uint(v) >> 23) & 255u) - 127;
+  const int f = 7 - e;
+  return f > 120 ? 120 : (f < -120 ? -120 : f);
+}
 
 // byte offset of 16-byte chunk c of row r in a 128-byte-swizzled atom
 __host__ __device__ __forceinline__ uint32_t sw128(int r, int c) {
@@ -348,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNK; ++s) {
       mbar_init(&bars[kKFull + s], 1);
-      mbar_init(&bars[kKFree + s], kNumMma + 8);   // the MMA streams + both CTAs' four V warps
+      mbar_init(&bars[kKFree + s], kNumMma + 2);   // the MMA streams + both CTAs' V warps
       mbar_init(&bars[kKPeerFull + s], 1);
       mbar_init(&bars[kScL + s], 1);
     }
@@ -358,8 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[kPReady + s], 16);
-      mbar_init(&bars[kVReady + s], 8);
+      mbar_init(&bars[kVReady + s], 2);         // one V warp per CTA
       mbar_init(&bars[kPvDone + s], kNumMma);
+      mbar_init(&bars[kVFull + s], 1);          // plus 16 KB of copies
     }
     for (int s = 0; s < kNSc; ++s) mbar_init(&bars[kScR + s], 1);
     mbar_init(&bars[kQReady], 2);
@@ -478,13 +510,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && first && item > 0) ok = wait_bar(&bars[kOFree], (item - 1) & 1);
         if (!ok) return;
         tc_fence_after();
-        const uint64_t pa = smem_desc(sp + (jj % kNP) * kPBuf, 16, 1024, 2);
+        // A: P, one K-major tile per term (rows of 64 token codes, 64-byte
+        // swizzle); B: the value codes, MN-major, 8-token groups of 1 KB
+        const uint64_t pa = smem_desc(sp + (jj % kNP) * kPBuf, 16, 512, 4);
         if (k < 2) {
-          const uint64_t va = smem_desc(sv + x * kVBuf + k * kVHalf, 1024, 2048, 2);
+          const uint64_t va = smem_desc(sv + x * kVBuf + k * kVHalf, kVHalf, 1024, 2);
 #pragma unroll
-          for (int ks = 0; ks < kBlk / 16; ++ks)
-            umma_pair_f16(tbase + 128 * k, pa + ((ks * 32) >> 4), va + ((ks * 4096) >> 4),
-                          kIdescPV, (first && ks == 0) ? 0u : 1u);
+          for (int ks = 0; ks < kBlk / 32; ++ks)
+#pragma unroll
+            for (int t = 0; t < kPTerms; ++t)
+              umma_pair_f8(tbase + 128 * k, pa + ((t * kPTerm + 32 * ks) >> 4),
+                           va + ((ks * 4096) >> 4), kIdescPV,
+                           (first && ks == 0 && t == 0) ? 0u : 1u);
         }
         umma_commit_pair(&bars[kPvDone + x]);   // frees V buffer x and P buffer jj % 2
       };
@@ -514,94 +551,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit_pair_local(&bars[kDrain + k]);
       mbar_wait_cluster(&bars[kDrain + k], 0);
     }
-  } else if (warp >= kWarpV) {
-    // ---------------- V conversion: E4M3 codes -> f16 B operand of PV ----------------
-    const int vt = threadIdx.x - 32 * kWarpV;             // 0..127
-    const int tt = vt & 63, vh = vt >> 6;                 // token, PV half
-    const int row = tt & 31;
-    // Token tt sits in the key stage of CTA tt / 32.  PV half h covers value
-    // dims 256h + [0, 256); this CTA holds dims 256h + 128*rank + [0, 128),
-    // the stage's 128-dim atom 2h + rank.  This thread converts half vh.
-    const uint32_t src = mapa_shared(smem_u32(smem + kOffK), static_cast<uint32_t>(tt >> 5)) +
-                         (2 * vh + rank) * kQkAtom;
+  } else if (warp == kWarpV) {
+    // ---------------- token scales and value copies ----------------
+    // Per block: the token scales for the softmax (0 past the end of the
+    // sequence or off the cache) and their maximum, first, so the softmax
+    // never waits for the copies.  Then, once the block's key stages have
+    // landed in both CTAs and value buffer x is free in both, lane 0 copies
+    // the raw code atoms of this CTA's 32 tokens into both CTAs' buffers:
+    // PV half k covers value dims 256k + [0, 256), of which CTA r holds
+    // 256k + 128r + [0, 128), key-stage atom 2k + r of either CTA; this CTA's
+    // tokens are rows 32*rank + [0, 32) of every buffer.
     const float* kscl = reinterpret_cast<const float*>(smem + kOffKSc);
     float* ring = reinterpret_cast<float*>(smem + kOffScR);
-    int32_t j = 0;
+    float* ring_max = reinterpret_cast<float*>(smem + kOffScMax);
+    int32_t j = 0, pending = -1;   // a block whose copies into this CTA were not waited for
     bool ok = true;
     for_pieces(p, u0, u1, [&](int b, int32_t t0, int32_t nt) {
       const int32_t ntok = seq_tokens(p, b);
       for (int32_t i = 0; i < nt; ++i, ++j) {
-        const int s = j % kNK, x = j & 1;
+        const int s = j % kNK, x = j & 1, e = j & (kNSc - 1);
         const uint32_t n = static_cast<uint32_t>(j / kNK);
-        // both CTAs' stages have landed: the leader's barrier counts both
-        // loads, and the leader's first V thread forwards its completion (off
-        // the MMA streams, which a remote arrive would hold up)
-        ok = ok && wait_bar(&bars[rank == 0 ? kKFull + s : kKPeerFull + s], n & 1u);
-        if (rank == 0 && vt == 0 && ok)
-          mbar_arrive_remote(mapa_shared(smem_u32(&bars[kKPeerFull + s]), 1));
-        ok = ok && wait_bar(&bars[kScL + s], n & 1u);
         const int32_t nvalid = min(kBlk, ntok - (t0 + i) * kBlk);
-        if (vt < 32) {
-          // token scales for the softmax first (0 past the end or off the
-          // cache), so the softmax never waits for the conversion below
-          if (ok) {
-            const bool in = flag[s] != 0;
-            const float2 sv = reinterpret_cast<const float2*>(kscl + s * kBlk)[vt];
-            reinterpret_cast<float2*>(ring + (j & (kNSc - 1)) * kBlk)[vt] =
-                make_float2(in && 2 * vt < nvalid ? sv.x : 0.0f, in && 2 * vt + 1 < nvalid ? sv.y : 0.0f);
+        ok = ok && wait_bar(&bars[kScL + s], n & 1u);
+        if (ok) {
+          const bool in = flag[s] != 0;
+          const float2 sv = reinterpret_cast<const float2*>(kscl + s * kBlk)[lane];
+          const float s0 = in && 2 * lane < nvalid ? sv.x : 0.0f;
+          const float s1 = in && 2 * lane + 1 < nvalid ? sv.y : 0.0f;
+          reinterpret_cast<float2*>(ring + e * kBlk)[lane] = make_float2(s0, s1);
+          float mx = fmaxf(s0, s1);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          if (lane == 0) ring_max[e] = mx;
+        }
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(&bars[kScR + e]);
+        // both CTAs' stages have landed: the leader's barrier counts both
+        // loads, and the leader forwards its completion
+        ok = ok && wait_bar(&bars[rank == 0 ? kKFull + s : kKPeerFull + s], n & 1u);
+        if (rank == 0 && lane == 0 && ok)
+          mbar_arrive_remote(mapa_shared(smem_u32(&bars[kKPeerFull + s]), 1));
+        // buffer x is free in both CTAs once PV(j - 2) has completed
+        if (j >= 2) ok = ok && wait_bar(&bars[kPvDone + x], ((j >> 1) & 1) ^ 1);
+        if (lane == 0 && ok) {
+          mbar_arrive_expect_tx(&bars[kVFull + x], kVBuf);   // own two atoms + the peer's two
+          const uint8_t* st = smem + kOffK + s * kStage;
+          const uint32_t dst = smem_u32(smem + kOffV + x * kVBuf) + rank * kQkAtom;
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (uint32_t r = 0; r < 2; ++r)
+              bulk_copy_to_cluster(mapa_shared(dst + k * kVHalf, r), st + (2 * k + r) * kQkAtom,
+                                   kQkAtom, mapa_shared(smem_u32(&bars[kVFull + x]), r));
+          pending = j;
+        }
+        ok = ok && wait_bar(&bars[kVFull + x], (j >> 1) & 1);
+        if (ok) pending = -1;
+        // rows past the end of the sequence may hold any codes, NaN patterns
+        // among them, which a zero probability would not cancel
+        if (ok && nvalid < kBlk) {
+          uint8_t* vb = smem + kOffV + x * kVBuf;
+          const int nrow = kBlk - nvalid;
+          for (int idx = lane; idx < 2 * nrow * 8; idx += 32) {
+            const int k = idx / (nrow * 8), rr = idx - k * nrow * 8;
+            *reinterpret_cast<uint4*>(vb + k * kVHalf + (nvalid + (rr >> 3)) * 128 + (rr & 7) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
           }
-          __syncwarp();
-          if (vt == 0 && ok) mbar_arrive(&bars[kScR + (j & (kNSc - 1))]);
+          fence_proxy_async_smem();
         }
-        // Load and convert the codes into registers, then hand the key stage
-        // back at once; only the stores wait for the converted-V buffer.
-        const bool valid = ok && tt < nvalid;
-        const uint32_t sa = src + s * kStage;
-        uint4 wv[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          wv[c] = valid ? ld_cluster128(sa + sw128(row, c)) : make_uint4(0, 0, 0, 0);
-        uint32_t f[8][8];                                 // values * 2^-8 (undone in the epilogue)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {                     // 16 codes = dims 16c..16c+15
-          e4m3x4_to_f16x2x2_shr8(wv[c].x, f[c][0], f[c][1]);
-          e4m3x4_to_f16x2x2_shr8(wv[c].y, f[c][2], f[c][3]);
-          e4m3x4_to_f16x2x2_shr8(wv[c].z, f[c][4], f[c][5]);
-          e4m3x4_to_f16x2x2_shr8(wv[c].w, f[c][6], f[c][7]);
-        }
-        // The OR reads every loaded register and its result is stored, so the
-        // store, and the arrivals issued after it, wait until this thread's
-        // loads from both stages have returned; the warp sync covers all lanes.
-        uint32_t dep = 0;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) dep |= wv[c].x | wv[c].y | wv[c].z | wv[c].w;
-        st_shared_keep(smem_u32(smem + kOffSink) + 4 * (warp - kWarpV), dep);
         __syncwarp();
         if (lane == 0 && ok) {
+          arrive_leader(&bars[kVReady + x], rank);
+          // the copies out of this CTA's stage have landed in both CTAs
           mbar_arrive(&bars[kKFree + s]);
           mbar_arrive_remote(mapa_shared(smem_u32(&bars[kKFree + s]), rank ^ 1u));
         }
-        if (j >= 2) ok = ok && wait_bar(&bars[kPvDone + x], ((j >> 1) & 1) ^ 1);
-        if (ok) {
-          // MN-major, 128-byte swizzle: atoms of 64 dims x 8 tokens (1 KB),
-          // two atoms per 8 tokens
-          uint8_t* dst = smem + kOffV + x * kVBuf + vh * kVHalf;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {              // 8 dims per 16-byte V chunk
-              const int cc = 2 * c + hh;
-              const uint32_t off = (cc >> 3) * 1024 + (tt >> 3) * 2048 + (tt & 7) * 128 +
-                                   (((cc & 7) ^ (tt & 7)) << 4);
-              *reinterpret_cast<uint4*>(dst + off) = make_uint4(
-                  f[c][4 * hh], f[c][4 * hh + 1], f[c][4 * hh + 2], f[c][4 * hh + 3]);
-            }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && ok) arrive_leader(&bars[kVReady + x], rank);   // per warp
       }
     });
+    // copies into this CTA after a wait that gave up land before the CTA exits
+    if (lane == 0 && pending >= 0)
+      mbar_wait_cluster(&bars[kVFull + (pending & 1)], (pending >> 1) & 1);
   } else {
     // ---------------- softmax warps: scores, P, epilogue ----------------
     // Eight warps.  Warp w reads TMEM lane quarter q = w % 4 (lane L = 32q +
@@ -617,6 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tbase + (static_cast<uint32_t>(32 * q4) << 16);
     const float* qexp = reinterpret_cast<const float*>(smem + kOffQ + 2 * kQPart);
     const float* ring = reinterpret_cast<const float*>(smem + kOffScR);
+    const float* ring_max = reinterpret_cast<const float*>(smem + kOffScMax);
     float* xm = reinterpret_cast<float*>(smem + kOffXm);
     float* xl = reinterpret_cast<float*>(smem + kOffXl);
     const float kNegInf = -__int_as_float(0x7f800000);
@@ -646,6 +676,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float alpha = p.sm_scale * kLog2e * qexp[hl];
 
       float m_ref = kNegInf, l_part = 0.0f;
+      int f_p = 0;              // P is stored as E4M3 terms of p * s * 2^f_p
+      bool f_set = false;       // f_p chosen (some block had p * s > 0)
       for (int32_t i = 0; i < nt; ++i, ++j) {
         const int s2 = j & 1, s3 = j % kNS;
         const int32_t nvalid = min(kBlk, ntok - (t0 + i) * kBlk);
@@ -672,8 +704,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 16; ++c) sacc[c] = 0.0f;
         }
         tc_fence_before();
-        // this thread's 16 token scales (0 past the end of the sequence or off the cache)
+        // this thread's 16 token scales (0 past the end of the sequence or off
+        // the cache) and the block's largest scale
         float sc[16];
+        const float smax = ring_max[j & (kNSc - 1)];
         {
           const float4* s4 = reinterpret_cast<const float4*>(ring + (j & (kNSc - 1)) * kBlk + 16 * part);
 #pragma unroll
@@ -706,13 +740,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && ok) arrive_leader(&bars[kSFree + s3], rank);
 #pragma unroll
         for (int o = 1; o < 4; ++o) bm = fmaxf(bm, xmj[((part + o) & 3) * 64 + hl]);
-        // Move the reference max when a score exceeds it by 2^8.  The vote keeps
-        // the TMEM accesses warp-uniform; the other three warps of these 32
-        // heads see the same head maxima and vote alike.
-        if (__any_sync(0xffffffffu, bm > m_ref + 8.0f)) {
-          const float m_new = fmaxf(m_ref, bm);
-          const float r = ex2(m_ref - m_new);             // 0 on the first block, 1 if unmoved
-          l_part *= r;
+        // Move the reference max when a score exceeds it by 2^8, and the
+        // power of two of P when this block's bound on p * s (its largest
+        // p, against the new reference, times its largest scale) would pass
+        // the E4M3 range at the current one; the new power puts the bound in
+        // [128, 256).  Either move rescales O.  The vote keeps the TMEM
+        // accesses warp-uniform; the other three warps of these 32 heads see
+        // the same head maxima and scales and decide alike.
+        const float m_new = bm > m_ref + 8.0f ? fmaxf(m_ref, bm) : m_ref;
+        const float vb = ex2(bm - m_new) * smax;
+        int f_new = f_p;
+        if (vb > 0.0f && (!f_set || vb * pow2f(f_p) > 448.0f)) f_new = pow2_exponent(vb);
+        if (__any_sync(0xffffffffu, m_new != m_ref || f_new != f_p)) {
+          const float rm = ex2(m_ref - m_new);            // 0 on the first block, 1 if unmoved
+          // before f is first set every P was 0, so O needs no power-of-two factor
+          const float r = f_set ? rm * pow2f(f_new) * pow2f(-f_p) : rm;
+          l_part *= rm;
           if (i > 0) {
             // O must not be in use by the previous block's PV
             ok = ok && wait_bar(&bars[kPvDone + ((j - 1) & 1)], ((j - 1) >> 1) & 1);
@@ -731,24 +774,39 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_wait_st();
             }
           }
-          m_ref = m_new;
         }
-        // ---- P (f16, token scale folded in) into the A operand of PV ----
-        uint32_t pk[8];
+        m_ref = m_new;
+        f_p = f_new;
+        f_set = f_set || vb > 0.0f;
+        // ---- P (token scale and 2^f folded in) as E4M3 terms: the A operand of PV ----
+        const float g = pow2f(f_p);
+        uint32_t pt[kPTerms][4] = {};
 #pragma unroll
         for (int c = 0; c < 16; c += 2) {
           const float p0 = ex2(x[c] - m_ref), p1 = ex2(x[c + 1] - m_ref);
           l_part += p0 + p1;
-          pk[c >> 1] = pack_f16x2(p0 * sc[c], p1 * sc[c + 1]);
+          float a0 = p0 * sc[c] * g, a1 = p1 * sc[c + 1] * g;
+#pragma unroll
+          for (int t = 0; t < kPTerms; ++t) {
+            const uint32_t code = f32x2_to_e4m3x2(a0, a1);
+            pt[t][c >> 2] |= code << (16 * ((c >> 1) & 1));
+            if (t + 1 < kPTerms) {                        // the residual for the next term
+              const uint32_t hf = e4m3x2_to_f16x2(code);
+              a0 -= __half2float(__ushort_as_half(static_cast<uint16_t>(hf & 0xFFFFu)));
+              a1 -= __half2float(__ushort_as_half(static_cast<uint16_t>(hf >> 16)));
+            }
+          }
         }
         const int pb = j % kNP;
         if (j >= kNP)                                     // P buffer free: PV(j - 2) done
           ok = ok && wait_bar(&bars[kPvDone + pb], static_cast<uint32_t>((j >> 1) & 1) ^ 1u);
         if (ok) {
+          // term t, row hl: the codes of tokens 0-63, 16 per chunk
+          uint8_t* pbuf = smem + kOffP + pb * kPBuf;
 #pragma unroll
-          for (int k = 0; k < 2; ++k)
-            *reinterpret_cast<uint4*>(smem + kOffP + pb * kPBuf + sw128(hl, 2 * part + k)) =
-                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          for (int t = 0; t < kPTerms; ++t)
+            *reinterpret_cast<uint4*>(pbuf + t * kPTerm + sw64(hl, part)) =
+                make_uint4(pt[t][0], pt[t][1], pt[t][2], pt[t][3]);
         }
         tc_fence_before();
         fence_proxy_async_smem();
@@ -767,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float l_tot = l_part;
 #pragma unroll
         for (int o = 1; o < 4; ++o) l_tot += xl[((part + o) & 3) * 64 + hl];
-        const float inv = 256.0f / l_tot;                 // V was converted as V * 2^-8
+        const float inv = pow2f(-f_p) / l_tot;            // P was stored times 2^f_p
         const int hg = 64 * static_cast<int>(rank) + hl;
         const int64_t slot = pair + b;
         float* orow = p.ws_o + (slot * kHq + hg) * kDv;

@@ -352,6 +352,18 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       : "memory");
 }
 
+// 1-D bulk copy from this CTA's shared memory to the shared memory of a CTA
+// of the cluster (this one included), completed on an mbarrier of the
+// destination CTA: dst and bar are shared::cluster addresses (from mapa).
+// 16-byte aligned, size % 16 == 0.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, const void* smem_src,
+                                                     uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "r"(smem_u32(smem_src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Tensor memory (tcgen05) for a CTA pair
 // ---------------------------------------------------------------------------

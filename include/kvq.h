@@ -220,11 +220,13 @@ size_t kvq_decode_workspace_size(const kvq_cache* cache, int32_t B, int32_t num_
  * {64, 128} with separate V pages, ps a multiple of 16 and
  * num_q_heads / Hkv <= 16; or Dk = 576, Dv = 512 with V aliasing K, one KV
  * head, 128 query heads, TOKEN scales and ps a multiple of 64.  The second
- * shape runs on the tensor cores: each query row is scaled by a power of
- * two to a maximum in [128, 256) and split into two E4M3 terms (any BF16
- * range; exact for scaled elements of magnitude >= 2^-2, smaller ones are
- * rounded at the E4M3 step 2^-9), and the E4M3 NaN
- * codes 0x7F / 0xFF, which kvq_append never writes, read as +-480 there.
+ * shape runs on the tensor cores on the stored codes: each query row is
+ * scaled by a power of two to a maximum in [128, 256) and split into two
+ * E4M3 terms (any BF16 range; exact for scaled elements of magnitude >= 2^-2,
+ * smaller ones are rounded at the E4M3 step 2^-9); the probabilities, times
+ * the token scales and a power of two per head, into three (about 2^-12
+ * relative); and an E4M3 NaN code (0x7F / 0xFF, which
+ * kvq_append never writes) in a cached token gives NaN there.
  * The kernels are launched as programmatic dependents of the previous work
  * on the stream.  The 8-head kernel reads seq_lens and block_table to plan
  * its split while that work may still run (the kernel launched just before
