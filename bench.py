@@ -876,11 +876,61 @@ def run_ours(args):
                                                   e2e=(name == "gqa"), bf16=(name != "wide"))
         s = W.spec_by_name("gqa")
         line["bulk_append"] = run_bulk_append(s, dev, stream)
+        if world == 1:
+            line["concurrency"] = run_concurrency(args, dev, stream)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def decode_call_at(B, dt, args, dev, stream, hbm):
+    """Decode-call time on the gqa shape (64 query / 8 KV heads, d 128, page
+    16) with B sequences of 8,192 tokens in cache format dt: CUDA graphs of
+    REPS back-to-back calls, events around every replay.  Returns the timing
+    record and the cache bytes per token of the allocated pages."""
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch
+    spec = W.spec_by_name("gqa")
+    spec.seq_lens = [8192] * B
+    spec.kv_dtype = dt
+    wl = W.make_workload(spec, seed=0, device=dev)
+    db = DecodeBatch(wl, device=dev)
+    db.prefill()
+    c = db.cache
+    nbytes = sum(x.numel() * x.element_size() for x in
+                 (c.k_pages, c.v_pages, c.k_scale, c.v_scale) if x is not None)
+    per_token = nbytes / (wl.num_pages * spec.page_size)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            db.decode(use_abort=False, stream=stream)
+        gd = capture(lambda: [db.decode(use_abort=False, stream=stream)
+                              for _ in range(REPS)], stream)
+        for _ in range(3):
+            gd.replay()
+        t = stats(time_replays(gd.replay, stream, args.min_seconds) / REPS)
+    kv = wl.kv_bytes_read()               # bytes of this cache format
+    rec = {"ms": t, "kv_gbs": kv / (t["mean"] * 1e-3) / 1e9,
+           "frac_of_hbm": kv / (t["mean"] * 1e-3) / 1e9 / hbm,
+           "decode_tokens_per_s": B / (t["mean"] * 1e-3)}
+    del gd, db
+    torch.cuda.empty_cache()
+    return rec, per_token
+
+
+def run_concurrency(args, dev, stream):
+    """FP8 decode call at low concurrency (B = 1, 8, 16 sequences of 8,192
+    tokens, gqa shape), each after the same idle time as the carried batches."""
+    from fp8_kv_paged_kvq_b200 import workloads as W
+    hbm, _ = peaks()
+    out = {"workload": "gqa shape, B x 8,192 tokens, FP8 head scales, decode call only",
+           "timing": f"CUDA graphs of {REPS} back-to-back calls, >= {args.min_seconds} s each, "
+                     f"after {args.idle_seconds} s idle"}
+    for B in (1, 8, 16):
+        time.sleep(args.idle_seconds)
+        out[f"B{B}"], _ = decode_call_at(B, W.FP8, args, dev, stream, hbm)
+    return out
 
 
 def run_sweep(args):
@@ -892,7 +942,6 @@ def run_sweep(args):
     torch.cuda.set_device(dev)
     from fp8_kv_paged_kvq_b200 import build as kvq_build
     from fp8_kv_paged_kvq_b200 import workloads as W
-    from fp8_kv_paged_kvq_b200.pipeline import DecodeBatch
     kvq_build.build()
     stream = torch.cuda.Stream(device=dev)
     hbm, _ = peaks()
@@ -902,28 +951,7 @@ def run_sweep(args):
     for B in (1, 8, 16, 32, 64):
         row = {"B": B}
         for dt in (W.FP8, W.BF16):
-            spec = W.spec_by_name("gqa")
-            spec.seq_lens = [8192] * B
-            spec.kv_dtype = dt
-            wl = W.make_workload(spec, seed=0, device=dev)
-            db = DecodeBatch(wl, device=dev)
-            db.prefill()
-            c = db.cache
-            nbytes = sum(x.numel() * x.element_size() for x in
-                         (c.k_pages, c.v_pages, c.k_scale, c.v_scale) if x is not None)
-            per_token[dt] = nbytes / (wl.num_pages * spec.page_size)
-            with torch.cuda.stream(stream):
-                for _ in range(3):
-                    db.decode(use_abort=False, stream=stream)
-                gd = capture(lambda: [db.decode(use_abort=False, stream=stream)
-                                      for _ in range(REPS)], stream)
-                t = stats(time_replays(gd.replay, stream, args.min_seconds) / REPS)
-            kv = wl.kv_bytes_read()               # bytes of this cache format
-            row[dt] = {"ms": t, "kv_gbs": kv / (t["mean"] * 1e-3) / 1e9,
-                       "frac_of_hbm": kv / (t["mean"] * 1e-3) / 1e9 / hbm,
-                       "decode_tokens_per_s": B / (t["mean"] * 1e-3)}
-            del gd, db
-            torch.cuda.empty_cache()
+            row[dt], per_token[dt] = decode_call_at(B, dt, args, dev, stream, hbm)
         row["fp8_over_bf16_time"] = row[W.FP8]["ms"]["mean"] / row[W.BF16]["ms"]["mean"]
         rows.append(row)
     line = {"sweep": "gqa shape, 8,192 tokens per sequence, decode call only",
