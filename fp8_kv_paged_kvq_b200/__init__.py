@@ -77,10 +77,11 @@ def lib() -> ctypes.CDLL:
         L.kvq_e4m3_encode_bits.argtypes = [_U32, _U32, _VP, _VP]
         L.kvq_e4m3_quantize_bits.argtypes = [_U32, _U32, ctypes.c_float, _VP, _VP]
         L.kvq_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+        L.kvq_wait_timeout_check.argtypes = [_VP, _VP]
         for f in ("kvq_amax", "kvq_scale_from_amax", "kvq_append", "kvq_validate", "kvq_decode",
                   "kvq_decode_bf16", "kvq_decode_noalloc", "kvq_e4m3_encode_bits",
                   "kvq_e4m3_quantize_bits",
-                  "kvq_device_error"):
+                  "kvq_device_error", "kvq_wait_timeout_check"):
             getattr(L, f).restype = _I32
         _lib = L
     return _lib
@@ -274,6 +275,11 @@ def e4m3_quantize_bits(start: int, count: int, scale: float,
            lib().kvq_e4m3_quantize_bits(start, count, ctypes.c_float(scale), _ptr(out),
                                         _stream(stream)))
     return out
+
+
+def wait_timeout_check(timed_out: torch.Tensor, stream=None) -> None:
+    """Run the bounded-wait check kernel (about one second); see kvq_wait_timeout_check."""
+    _check("kvq_wait_timeout_check", lib().kvq_wait_timeout_check(_ptr(timed_out), _stream(stream)))
 
 
 def device_error() -> int:

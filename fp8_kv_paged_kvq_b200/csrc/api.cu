@@ -301,6 +301,12 @@ kvq_status kvq_e4m3_encode_bits(uint32_t start, uint32_t count, uint8_t* out, vo
   return from_cuda(launch_encode_bits(start, count, out, static_cast<cudaStream_t>(stream)));
 }
 
+kvq_status kvq_wait_timeout_check(int32_t* timed_out, void* stream) {
+  if (timed_out == nullptr || (reinterpret_cast<uintptr_t>(timed_out) & 3u))
+    return KVQ_ERR_INVALID_ARG;
+  return from_cuda(launch_wait_timeout_check(timed_out, static_cast<cudaStream_t>(stream)));
+}
+
 kvq_status kvq_device_error(uint32_t* flags_host) {
   if (flags_host == nullptr) return KVQ_ERR_INVALID_ARG;
   return from_cuda(read_and_clear_error_flags(flags_host));

@@ -34,6 +34,7 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
                             int32_t B, int32_t max_pages, uint8_t* abort_mask,
                             int32_t* n_aborted, int32_t* first_bad, cudaStream_t stream);
 cudaError_t read_and_clear_error_flags(uint32_t* flags);
+cudaError_t launch_wait_timeout_check(int32_t* timed_out, cudaStream_t stream);
 
 // Ask for the largest shared-memory carveout for `kernel` on the current
 // device (once per device).  The tag check and the wide pre-pass, which run

@@ -401,6 +401,23 @@ cudaError_t launch_validate(const uint32_t* tags, int32_t P, const int32_t* bloc
                             max_pages, abort_mask, n_aborted, first_bad);
 }
 
+// One thread waits, through the decode kernels' bounded mbarrier wait, on a
+// barrier that nothing completes: after the wait's limit (about one second)
+// it records kErrWaitTimeout, and the kernel writes 1 to *timed_out (0 if
+// the wait had returned true).
+__global__ void wait_timeout_check_kernel(int32_t* timed_out) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  *timed_out = mbar_wait(&bar, 0) ? 0 : 1;
+}
+
+cudaError_t launch_wait_timeout_check(int32_t* timed_out, cudaStream_t stream) {
+  wait_timeout_check_kernel<<<1, 32, 0, stream>>>(timed_out);
+  return cudaGetLastError();
+}
+
 cudaError_t read_and_clear_error_flags(uint32_t* flags) {
   uint32_t zero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(flags, g_error_flags, sizeof(uint32_t));

@@ -308,6 +308,17 @@ kvq_status kvq_e4m3_quantize_bits(uint32_t start, uint32_t count, float scale, u
  */
 kvq_status kvq_device_error(uint32_t* flags_host);
 
+/*
+ * Exercises the error path above: one thread waits, through the bounded
+ * mbarrier wait the decode kernels use, on a barrier that nothing
+ * completes.  After the wait's limit (about one second) the kernel sets bit
+ * 0 of the error word and writes 1 to *timed_out (device i32, 4-byte
+ * aligned; 0 would mean the wait returned normally).  The context stays
+ * usable; read kvq_device_error afterwards to see and clear the bit, since
+ * the tensor-core decode kernel's waits give up at once while it is set.
+ */
+kvq_status kvq_wait_timeout_check(int32_t* timed_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
