@@ -100,6 +100,7 @@ struct GqaParams {
   float* out;
   float* lse;
   int32_t* ws_pre;   // [B+2] unit prefix, then the count of working CTAs (written by CTA 0)
+  int32_t* ws_bounds;  // [num_ctas+1] first unit of each working CTA, then U
   float* ws_lse;     // [slots][G]
   float* ws_o;       // [slots][G][Dv]
   int32_t num_ctas;
@@ -115,33 +116,81 @@ __device__ __forceinline__ int32_t seq_tokens(const GqaParams& p, int b, bool us
   return static_cast<int32_t>(n > cap ? cap : n);
 }
 
-// Exclusive prefix over b of Hkv * ceil(tokens_b / 16) into pre[0..B]: each
-// thread sums a run of sequences, a warp scan and the warps' totals give
-// each run its start.  Called by all threads of the block; scratch holds one
-// int per warp.
-__device__ void block_prefix_units(const GqaParams& p, int32_t* pre, int32_t* scratch,
-                                   bool use_abort) {
+// Each (sequence, KV head) segment with tiles also carries kPieceCost
+// virtual units in the split: a piece ends with the warps' merge and the
+// partial's write, and the next one starts with its query and scale loads,
+// about as long as this many tiles take to stream.  Without them a CTA whose
+// range crosses many short segments ends well after the others.
+constexpr int32_t kPieceCost = 48;
+
+// Exclusive prefixes over b of Hkv * tiles_b (pre[0..B], the units) and of
+// Hkv * (tiles_b + kPieceCost if tiles_b > 0) (wpre[0..B], the weighted units
+// the split divides), tiles_b = ceil(tokens_b / 16): each thread sums a run of
+// sequences, a warp scan and the warps' totals give each run its start.
+// Called by all threads of the block; scratch holds two ints per warp.
+__device__ void block_prefix_units(const GqaParams& p, int32_t* pre, int32_t* wpre,
+                                   int32_t* scratch, bool use_abort) {
   const int nthr = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = nthr >> 5;
   const int per = (p.B + nthr - 1) / nthr;
   const int lo = min(p.B, tid * per), hi = min(p.B, lo + per);
-  int32_t sum = 0;
-  for (int b = lo; b < hi; ++b) sum += p.c.Hkv * ((seq_tokens(p, b, use_abort) + 15) >> 4);
-  int32_t incl = sum;
+  auto units = [&](int b) { return p.c.Hkv * ((seq_tokens(p, b, use_abort) + 15) >> 4); };
+  int32_t sum = 0, wsum = 0;
+  for (int b = lo; b < hi; ++b) {
+    const int32_t x = units(b);
+    sum += x;
+    wsum += x > 0 ? x + p.c.Hkv * kPieceCost : 0;
+  }
+  int32_t incl = sum, wincl = wsum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
+    const int32_t wv = __shfl_up_sync(0xffffffffu, wincl, o);
+    if (lane >= o) {
+      incl += v;
+      wincl += wv;
+    }
   }
-  if (lane == 31) scratch[warp] = incl;
+  if (lane == 31) {
+    scratch[warp] = incl;
+    scratch[nw + warp] = wincl;
+  }
   __syncthreads();
-  int32_t run = incl - sum;
-  for (int w = 0; w < warp; ++w) run += scratch[w];
+  int32_t run = incl - sum, wrun = wincl - wsum;
+  for (int w = 0; w < warp; ++w) {
+    run += scratch[w];
+    wrun += scratch[nw + w];
+  }
   for (int b = lo; b < hi; ++b) {
     pre[b] = run;
-    run += p.c.Hkv * ((seq_tokens(p, b, use_abort) + 15) >> 4);
+    wpre[b] = wrun;
+    const int32_t x = units(b);
+    run += x;
+    wrun += x > 0 ? x + p.c.Hkv * kPieceCost : 0;
   }
-  if (tid == nthr - 1) pre[p.B] = run;      // the last run ends at B
+  if (tid == nthr - 1) {                    // the last run ends at B
+    pre[p.B] = run;
+    wpre[p.B] = wrun;
+  }
   __syncthreads();
+}
+
+// First real unit at or after weighted position w (0 <= w <= wpre[B]): in
+// sequence b each of its Hkv segments spans tiles_b + kPieceCost weighted
+// units, the virtual ones first.
+__device__ __forceinline__ int32_t real_unit(const GqaParams& p, const int32_t* pre,
+                                             const int32_t* wpre, int64_t w) {
+  if (w >= wpre[p.B]) return pre[p.B];
+  int lo = 0, hi = p.B;                     // largest b with wpre[b] <= w (a sequence with tiles)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (wpre[mid] <= w) lo = mid; else hi = mid;
+  }
+  const int32_t tiles = (pre[lo + 1] - pre[lo]) / p.c.Hkv;
+  const int32_t len = tiles + kPieceCost;
+  const int32_t off = static_cast<int32_t>(w - wpre[lo]);
+  const int32_t h = off / len, r = off - h * len;
+  return pre[lo] + h * tiles + max(0, r - kPieceCost);
 }
 
 // CTAs (or CTA pairs) that get units: at most num_ctas, at least min_units
@@ -209,7 +258,8 @@ struct GqaKernel {
   static constexpr int kOffMisc = kOffRedO + NW * kHeads * D * 4;   // flag, scratch
   static constexpr int kMiscInts = 4 + kThreads;
   static constexpr int kOffPre = kOffMisc + kMiscInts * 4;
-  static size_t smem_bytes(int B) { return 1024 + kOffPre + static_cast<size_t>(B + 1) * 4; }
+  // pre[B+1], then wpre[B+1]
+  static size_t smem_bytes(int B) { return 1024 + kOffPre + static_cast<size_t>(B + 1) * 8; }
 };
 
 // Registers: two CTAs per SM for one n-tile (128 per thread), and for the FP8
@@ -232,6 +282,7 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
   volatile int32_t* abort_flag = reinterpret_cast<int32_t*>(smem + K::kOffMisc);
   int32_t* scratch = reinterpret_cast<int32_t*>(smem + K::kOffMisc) + 4;
   int32_t* pre = reinterpret_cast<int32_t*>(smem + K::kOffPre);
+  int32_t* wpre = pre + p.B + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();                                 // the combine may launch (it waits for us)
@@ -252,20 +303,25 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
   const int cw = warp;
   int64_t U = 0, N = 0;
   int32_t u0 = 0, u1 = 0, kw = 0;
+  bool plain_split = false;                    // the plain c*U/N ranges
   auto plan = [&](bool use_abort) {
-    block_prefix_units(p, pre, scratch, use_abort);  // includes __syncthreads
+    block_prefix_units(p, pre, wpre, scratch, use_abort);  // includes __syncthreads
     U = pre[p.B];
     // Every sequence as long as the others (in tiles) and at least two CTAs
     // per segment: each segment gets the same number k >= 1 of CTAs, so CTA
     // boundaries fall on segment boundaries and no CTA holds two pieces.
-    // Otherwise (ragged batches, or one CTA per segment at most, where the
-    // idle CTAs would cost more than the extra pieces) the stream-K split.
+    // Equal lengths with fewer CTAs (where idle CTAs would cost more than the
+    // extra pieces): the stream-K split of the units, every CTA then holding
+    // one or two pieces.  Ragged batches: the stream-K split of the weighted
+    // units, each segment counting kPieceCost extra, so that a CTA whose
+    // range crosses many short segments gets fewer tiles.
     const int32_t t0 = p.B > 0 ? pre[1] - pre[0] : 0;
     int uneven = 0;
     for (int b = threadIdx.x; b < p.B; b += blockDim.x) uneven |= (pre[b + 1] - pre[b]) != t0;
     uneven = __syncthreads_or(uneven);
     const int64_t segs = static_cast<int64_t>(p.B) * p.c.Hkv;
-    if (!uneven && t0 > 0 && 2 * segs <= p.num_ctas) {
+    const bool aligned = !uneven && t0 > 0 && 2 * segs <= p.num_ctas;
+    if (aligned) {
       const int64_t tseg = U / segs;               // tiles of one segment
       int64_t k = p.num_ctas / segs;
       const int64_t kmax = tseg / kMinTilesPerCta;
@@ -275,8 +331,15 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
       N = working_ctas(p.num_ctas, U, kMinTilesPerCta);
     }
     const bool works = static_cast<int64_t>(blockIdx.x) < N;
-    u0 = works ? static_cast<int32_t>(U * blockIdx.x / N) : 0;
-    u1 = works ? static_cast<int32_t>(U * (blockIdx.x + 1) / N) : 0;
+    plain_split = !uneven;                    // c*U/N, no weights
+    if (!uneven) {
+      u0 = works ? static_cast<int32_t>(U * blockIdx.x / N) : 0;
+      u1 = works ? static_cast<int32_t>(U * (blockIdx.x + 1) / N) : 0;
+    } else {                                    // equal shares of the weighted units
+      const int64_t W = wpre[p.B];
+      u0 = works ? real_unit(p, pre, wpre, W * blockIdx.x / N) : 0;
+      u1 = works ? real_unit(p, pre, wpre, W * (blockIdx.x + 1) / N) : 0;
+    }
     // warp cw takes the CTA's tiles n = cw + NW*k, k = 0 .. kw-1
     const int32_t n_cta = u1 - u0;
     kw = n_cta > cw ? (n_cta - cw + NW - 1) / NW : 0;
@@ -314,8 +377,15 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
   }
   if (blockIdx.x == 0) {
     for (int b = threadIdx.x; b <= p.B; b += blockDim.x) p.ws_pre[b] = pre[b];
-    if (threadIdx.x == 0) p.ws_pre[p.B + 1] = static_cast<int32_t>(N);
+    // N, negated when the split is the weighted one (the combine then looks
+    // the pieces up in the CTAs' starts rather than in c*U/N)
+    if (threadIdx.x == 0) {
+      p.ws_pre[p.B + 1] = plain_split ? static_cast<int32_t>(N) : -static_cast<int32_t>(N);
+      p.ws_bounds[N] = static_cast<int32_t>(U);
+    }
   }
+  // where this CTA's units start, for the combine's piece lookup
+  if (threadIdx.x == 0 && static_cast<int64_t>(blockIdx.x) < N) p.ws_bounds[blockIdx.x] = u0;
   if (u0 >= u1) return;                          // no units: nothing issued, nothing to wait on
 
   // ---------------- this warp's pipeline ----------------
@@ -671,6 +741,7 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
 // ---------------------------------------------------------------------------
 struct CombineParams {
   const int32_t* ws_pre;
+  const int32_t* ws_bounds;   // first unit of each working CTA (then U), or null: c*U/N
   const float* ws_lse;
   const float* ws_o;
   int32_t B, Hkv, G, Hq, Dv, heads_per_block, lanes_log2;
@@ -683,6 +754,7 @@ constexpr int kCombOutputs = 2048;    // outputs per block (heads_per_block * Dv
 constexpr int kCombMaxThreads = kCombOutputs / 4;   // threads per block at most
 constexpr int kCombGroup = 4;         // pieces per round of loads
 constexpr int kCombMaxLanesLog2 = 3;  // at most 8 sub-lanes per group of four outputs
+constexpr int kCombMaxBounds = 2048;  // CTA starts staged in shared memory at most
 
 // CTA of a launch with N working CTAs over U units that owns unit u.
 __device__ __forceinline__ int64_t owner_cta(int64_t u, int64_t N, int64_t U) {
@@ -732,9 +804,33 @@ __global__ void __launch_bounds__(kCombMaxThreads, 1) lse_combine_kernel(const C
   }
   // U >= tiles_b > 0 here
   const int64_t S = p.ws_pre[b] + static_cast<int64_t>(h) * tiles_b, E = S + tiles_b;
-  const int64_t N = p.ws_pre[p.B + 1];          // the decode launch's working CTAs
-  const int64_t cs = owner_cta(S, N, U);
-  const int np = static_cast<int>(owner_cta(E - 1, N, U) - cs + 1);
+  // the decode launch's working CTAs, negated after a weighted split
+  const int32_t nflag = p.ws_pre[p.B + 1];
+  const int64_t N = nflag < 0 ? -static_cast<int64_t>(nflag) : nflag;
+  const bool weighted = nflag < 0 && p.ws_bounds != nullptr;
+  // After a weighted split the CTAs' starts come into shared memory in one
+  // round of loads (when they fit) for the searches below.
+  __shared__ int32_t s_bounds[kCombMaxBounds];
+  const bool staged = weighted && N + 1 <= kCombMaxBounds;
+  if (staged) {
+    for (int i = threadIdx.x; i <= N; i += blockDim.x) s_bounds[i] = p.ws_bounds[i];
+    __syncthreads();
+  }
+  const int32_t* bounds = staged ? s_bounds : p.ws_bounds;
+  // CTA holding unit u: c*U/N's owner, or after a weighted split the last CTA
+  // whose range starts at or before u (a CTA with an empty range shares its
+  // start with the next one)
+  auto owner = [&](int64_t u) -> int64_t {
+    if (!weighted) return owner_cta(u, N, U);
+    int64_t lo = 0, hi = N;
+    while (hi - lo > 1) {
+      const int64_t mid = (lo + hi) >> 1;
+      if (bounds[mid] <= u) lo = mid; else hi = mid;
+    }
+    return lo;
+  };
+  const int64_t cs = owner(S);
+  const int np = static_cast<int>(owner(E - 1) - cs + 1);
   const int64_t slot0 = cs + seg;               // slot of piece k: slot0 + k
   // This sub-lane's pieces sub, sub + nl, ... (none for threads past the
   // block's outputs, which still take part in the shuffles), in groups of
@@ -827,11 +923,13 @@ __global__ void __launch_bounds__(kCombMaxThreads, 1) lse_combine_kernel(const C
 // ---------------------------------------------------------------------------
 // Host side: tensor maps, occupancy, dispatch
 // ---------------------------------------------------------------------------
-cudaError_t launch_lse_combine(const int32_t* ws_pre, const float* ws_lse, const float* ws_o,
-                               int32_t B, int32_t Hkv, int32_t G, int32_t Hq, int32_t Dv,
-                               int32_t num_ctas, float* out, float* lse, cudaStream_t stream) {
+cudaError_t launch_lse_combine(const int32_t* ws_pre, const int32_t* ws_bounds,
+                               const float* ws_lse, const float* ws_o, int32_t B, int32_t Hkv,
+                               int32_t G, int32_t Hq, int32_t Dv, int32_t num_ctas, float* out,
+                               float* lse, cudaStream_t stream) {
   CombineParams cp;
   cp.ws_pre = ws_pre;
+  cp.ws_bounds = ws_bounds;
   cp.ws_lse = ws_lse;
   cp.ws_o = ws_o;
   cp.B = B;
@@ -908,12 +1006,13 @@ static cudaError_t run_gqa(const DecodeArgs& a, const CUtensorMap& km, const CUt
   WorkspaceLayout wl = workspace_layout(a.B, a.c.Hkv, p.G, a.c.Dv, a.num_ctas);
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
   p.ws_pre = reinterpret_cast<int32_t*>(ws + wl.off_pre);
+  p.ws_bounds = reinterpret_cast<int32_t*>(ws + wl.off_bounds);
   p.ws_lse = reinterpret_cast<float*>(ws + wl.off_lse);
   p.ws_o = reinterpret_cast<float*>(ws + wl.off_o);
   e = launch_pdl(kern, dim3(a.num_ctas), dim3(K::kThreads), smem, a.stream, km, vm, p);
   if (e != cudaSuccess) return e;
-  return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, a.c.Hkv, p.G, a.Hq, a.c.Dv,
-                            a.num_ctas, a.out, a.lse, a.stream);
+  return launch_lse_combine(p.ws_pre, p.ws_bounds, p.ws_lse, p.ws_o, a.B, a.c.Hkv, p.G, a.Hq,
+                            a.c.Dv, a.num_ctas, a.out, a.lse, a.stream);
 }
 
 // Consumer warps and pipeline depth per configuration.

@@ -959,8 +959,8 @@ cudaError_t launch_wide_decode(const DecodeArgs& a, const CUtensorMap& kqk,
   cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, wide::wide_decode_kernel, kqk, ktail, p);
   if (e != cudaSuccess) return e;
-  return launch_lse_combine(p.ws_pre, p.ws_lse, p.ws_o, a.B, 1, wide::kHq, wide::kHq, wide::kDv,
-                            a.num_ctas, a.out, a.lse, a.stream);
+  return launch_lse_combine(p.ws_pre, nullptr, p.ws_lse, p.ws_o, a.B, 1, wide::kHq, wide::kHq,
+                            wide::kDv, a.num_ctas, a.out, a.lse, a.stream);
 }
 
 }  // namespace kvq

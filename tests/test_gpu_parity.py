@@ -536,6 +536,34 @@ def test_equal_tile_counts_split_on_segment_edges(num_ctas):
     assert kvq.device_error() == 0
 
 
+@pytest.mark.parametrize("num_ctas", [0, 1000])
+def test_weighted_split_with_ctas_inside_a_segments_start(num_ctas):
+    """A ragged batch (2,048 tiles and 1 tile on one KV head) with many CTAs:
+    the weighted split charges each segment 48 extra units at its start, so
+    with 1,000 CTAs the first CTAs' shares lie inside that charge and own no
+    tile; the combine must skip them when it looks up a segment's pieces."""
+    spec = W.Spec("weighted_empty", [32768, 16], 16, 8, 1, 128, 128, outlier_p=0.01)
+    wl, db, oc = build_both(spec, seed=22, num_ctas=num_ctas)
+    out, lse = db.step(check_tags=False)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), "weighted")
+    assert kvq.device_error() == 0
+
+
+def test_weighted_split_beyond_the_staged_starts():
+    """More than 2,047 working CTAs over a ragged batch (two long sequences on
+    two KV heads, 70,000 tiles, 2,100 CTAs): the combine searches the CTAs'
+    starts in global memory instead of staging them."""
+    spec = W.Spec("weighted_many_ctas", [300000, 260000], 16, 4, 2, 128, 128)
+    wl, db, oc = build_both(spec, seed=23, num_ctas=2100, canary=False)
+    out, lse = db.step(check_tags=False)
+    torch.cuda.synchronize()
+    ro, rl = OS.decode(wl, oc)
+    assert_decode_close(out, lse, ro.reshape(out.shape), rl.reshape(lse.shape), "many ctas")
+    assert kvq.device_error() == 0
+
+
 def test_many_short_segments_group_1():
     """32 KV heads with one query head each and 520 short ragged rows (1..60
     tokens, head dim 64): 16,640 segments, each CTA's range crossing about
