@@ -44,7 +44,7 @@
 namespace kvq {
 
 // Largest batch the decode kernels accept (the unit prefix lives in shared memory).
-constexpr int32_t kGqaMaxBatch = 8192;
+constexpr int32_t kGqaMaxBatch = 8000;   // three [B+1] arrays in shared memory
 
 // ---------------------------------------------------------------------------
 // Shared memory layout traits
@@ -127,9 +127,10 @@ constexpr int32_t kPieceCost = 48;
 // Hkv * (tiles_b + kPieceCost if tiles_b > 0) (wpre[0..B], the weighted units
 // the split divides), tiles_b = ceil(tokens_b / 16): each thread sums a run of
 // sequences, a warp scan and the warps' totals give each run its start.
-// Called by all threads of the block; scratch holds two ints per warp.
+// Also keeps each sequence's token count in ntok[b].  Called by all threads
+// of the block; scratch holds two ints per warp.
 __device__ void block_prefix_units(const GqaParams& p, int32_t* pre, int32_t* wpre,
-                                   int32_t* scratch, bool use_abort) {
+                                   int32_t* ntok, int32_t* scratch, bool use_abort) {
   const int nthr = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = nthr >> 5;
   const int per = (p.B + nthr - 1) / nthr;
@@ -164,6 +165,7 @@ __device__ void block_prefix_units(const GqaParams& p, int32_t* pre, int32_t* wp
   for (int b = lo; b < hi; ++b) {
     pre[b] = run;
     wpre[b] = wrun;
+    ntok[b] = seq_tokens(p, b, use_abort);
     const int32_t x = units(b);
     run += x;
     wrun += x > 0 ? x + p.c.Hkv * kPieceCost : 0;
@@ -222,7 +224,8 @@ struct Piece {
   int32_t ntok;         // tokens of the sequence
 };
 
-// Next piece starting at unit u (< u1).
+// Next piece starting at unit u (< u1).  pre is followed in shared memory
+// by the weighted prefix and the sequences' token counts (B+1 each).
 __device__ __forceinline__ Piece make_piece(const GqaParams& p, const int32_t* pre, int32_t u,
                                             int32_t u1, int32_t n0) {
   Piece pc;
@@ -234,7 +237,7 @@ __device__ __forceinline__ Piece make_piece(const GqaParams& p, const int32_t* p
   pc.nt = min(tiles_b - pc.t0, u1 - u);
   pc.seg = pc.b * p.c.Hkv + pc.h;
   pc.n0 = n0;
-  pc.ntok = seq_tokens(p, pc.b, true);
+  pc.ntok = pre[2 * (p.B + 1) + pc.b];
   return pc;
 }
 
@@ -257,9 +260,12 @@ struct GqaKernel {
   static constexpr int kOffRedO = kOffRedL + NW * kHeads * 4;
   static constexpr int kOffMisc = kOffRedO + NW * kHeads * D * 4;   // flag, scratch
   static constexpr int kMiscInts = 4 + kThreads;
-  static constexpr int kOffPre = kOffMisc + kMiscInts * 4;
-  // pre[B+1], then wpre[B+1]
-  static size_t smem_bytes(int B) { return 1024 + kOffPre + static_cast<size_t>(B + 1) * 8; }
+  // per-tensor or per-head scales of K and V, for up to kScaleHeads KV heads
+  static constexpr int kScaleHeads = 64;
+  static constexpr int kOffScales = kOffMisc + kMiscInts * 4;
+  static constexpr int kOffPre = kOffScales + 2 * kScaleHeads * 4;
+  // pre[B+1], wpre[B+1], ntok[B+1]
+  static size_t smem_bytes(int B) { return 1024 + kOffPre + static_cast<size_t>(B + 1) * 12; }
 };
 
 // Registers: two CTAs per SM for one n-tile (128 per thread), and for the FP8
@@ -283,6 +289,7 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
   int32_t* scratch = reinterpret_cast<int32_t*>(smem + K::kOffMisc) + 4;
   int32_t* pre = reinterpret_cast<int32_t*>(smem + K::kOffPre);
   int32_t* wpre = pre + p.B + 1;
+  int32_t* ntok = wpre + p.B + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();                                 // the combine may launch (it waits for us)
@@ -293,10 +300,11 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
   }
   if (lane == 0) { tma_prefetch_desc(&k_map); tma_prefetch_desc(&v_map); }
 
-  // The work plan.  Before the dependency wait the kernel reads only what no
-  // kernel of this library writes (sequence lengths and block-table entries)
-  // and writes nothing to global memory: it lays out the units as if no
-  // request were aborted and looks up its first pages.  After the wait it
+  // The work plan.  Before the dependency wait the kernel reads only what the
+  // kernel launched just before it does not write (sequence lengths,
+  // block-table entries, per-tensor or per-head scales) and writes nothing to
+  // global memory: it lays out the units as if no request were aborted and
+  // looks up its first pages.  After the wait it
   // reads the abort mask and redoes the plan only if some request aborted.
   // The units go to the first N CTAs, every one of which owns at least one
   // unit (the combine relies on it).
@@ -305,7 +313,7 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
   int32_t u0 = 0, u1 = 0, kw = 0;
   bool plain_split = false;                    // the plain c*U/N ranges
   auto plan = [&](bool use_abort) {
-    block_prefix_units(p, pre, wpre, scratch, use_abort);  // includes __syncthreads
+    block_prefix_units(p, pre, wpre, ntok, scratch, use_abort);  // includes __syncthreads
     U = pre[p.B];
     // Every sequence as long as the others (in tiles) and at least two CTAs
     // per segment: each segment gets the same number k >= 1 of CTAs, so CTA
@@ -361,6 +369,19 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
     }
   };
   int32_t cur_page, cur_hy, nxt_page, nxt_hy, batch0 = 0;
+  // Per-tensor or per-head scales into shared memory (made visible by the
+  // plan's barriers).  They are read before the dependency wait too: only
+  // kvq_scale_from_amax writes them, and it lets no kernel start before it
+  // ends.
+  if (FP8 && p.c.scale_mode <= 1 && p.c.Hkv <= K::kScaleHeads) {
+    float* sk = reinterpret_cast<float*>(smem + K::kOffScales);
+    const float* vs = p.c.v_pages ? p.c.v_scale : p.c.k_scale;
+    const int nh = p.c.scale_mode == 0 ? 1 : p.c.Hkv;
+    for (int i = threadIdx.x; i < nh; i += blockDim.x) {
+      sk[i] = p.c.k_scale[i];
+      sk[K::kScaleHeads + i] = vs[i];
+    }
+  }
   plan(false);
   lookup(0, cur_page, cur_hy);
   lookup(32, nxt_page, nxt_hy);
@@ -441,10 +462,16 @@ __global__ void __maxnreg__(NT == 1 ? (FP8 ? 120 : 128) : 255)
     // per-segment constants
     const int hk = pc.h;
     float alpha = p.sm_scale * kLog2e, vscale = 1.0f;
-    if (FP8) {
-      const float* vs = p.c.v_pages ? p.c.v_scale : p.c.k_scale;
-      if (p.c.scale_mode == 0) { alpha *= p.c.k_scale[0]; vscale = vs[0]; }
-      else if (p.c.scale_mode == 1) { alpha *= p.c.k_scale[hk]; vscale = vs[hk]; }
+    if (FP8 && p.c.scale_mode <= 1) {
+      const int i = p.c.scale_mode == 0 ? 0 : hk;
+      if (p.c.Hkv <= K::kScaleHeads) {
+        const float* sk = reinterpret_cast<const float*>(smem + K::kOffScales);
+        alpha *= sk[i];
+        vscale = sk[K::kScaleHeads + i];
+      } else {
+        alpha *= p.c.k_scale[i];
+        vscale = (p.c.v_pages ? p.c.v_scale : p.c.k_scale)[i];
+      }
     }
     // Q fragments (B operand of QK^T): head nt*8+g, dims k_dbase(j)..+3
     uint32_t qb[NT][L::kKSteps][2];

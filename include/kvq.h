@@ -216,7 +216,8 @@ size_t kvq_decode_workspace_size(const kvq_cache* cache, int32_t B, int32_t num_
  *               partial results are merged by a log-sum-exp combine launch.
  * Page ids outside [0, P) read as zeros (no fault); run kvq_validate first
  * to abort such requests instead.  Queries must lie within the FP16 range.
- * Requires cache->dtype == KVQ_FP8_E4M3.  Supported shapes: Dk == Dv in
+ * Requires cache->dtype == KVQ_FP8_E4M3 and B <= 8,000 (larger batches return
+ * KVQ_ERR_UNSUPPORTED).  Supported shapes: Dk == Dv in
  * {64, 128} with separate V pages, ps a multiple of 16 and
  * num_q_heads / Hkv <= 16; or Dk = 576, Dv = 512 with V aliasing K, one KV
  * head, 128 query heads, TOKEN scales and ps a multiple of 64.  The second
@@ -228,10 +229,12 @@ size_t kvq_decode_workspace_size(const kvq_cache* cache, int32_t B, int32_t num_
  * relative); and an E4M3 NaN code (0x7F / 0xFF, which
  * kvq_append never writes) in a cached token gives NaN there.
  * The kernels are launched as programmatic dependents of the previous work
- * on the stream.  The 8-head kernel reads seq_lens and block_table to plan
- * its split while that work may still run (the kernel launched just before
- * must not write them; kvq_validate and kvq_append never do) and everything
- * else, the abort mask included, after it has finished; the wide kernels
+ * on the stream.  The 8-head kernel reads seq_lens, block_table and the
+ * per-tensor or per-head scales to plan its split while that work may still
+ * run (the kernel launched just before must not write them; kvq_validate and
+ * kvq_append never do, and kvq_scale_from_amax lets no kernel start before
+ * it ends) and everything else, the abort mask included, after it has
+ * finished; the wide kernels
  * wait before reading any argument.  The last kernel of the call (the
  * log-sum-exp combine) lets the next kernel on the stream start once the
  * decode kernel has finished, while it still writes out and lse: a kernel
