@@ -12,12 +12,16 @@
 //
 //  * Work split.  The work units are 16-token tiles of one (sequence, KV
 //    head) segment, flattened in (b, h, tile) order after aborted and empty
-//    sequences are dropped.  Persistent CTA c takes units [c*U/N, (c+1)*U/N):
-//    every CTA gets the same number of tiles whatever the length mix, and a
-//    CTA's range covers at most a few segments ("pieces").  Each piece
-//    leaves one partial (o, lse) in the workspace at slot c + segment, which
-//    is unique because both c and the segment index grow along the unit
-//    order.  A combine launch merges the partials of each segment.
+//    sequences are dropped.  Persistent CTA c takes one contiguous range of
+//    units: [c*U/N, (c+1)*U/N) when all sequences have the same length (with
+//    N a multiple of the segments when there are CTAs enough, so that ranges
+//    start on segment edges), and for ragged batches equal shares of
+//    weighted units, each segment counting kPieceCost more, so that a CTA
+//    crossing many short segments gets fewer tiles.  A CTA's range covers a
+//    few segments ("pieces").  Each piece leaves one partial (o, lse) in the
+//    workspace at slot c + segment, which is unique because both c and the
+//    segment index grow along the unit order.  A combine launch merges the
+//    partials of each segment.
 //  * Pipeline.  Every warp streams its own tiles (n = warp + NW*k of the
 //    CTA's range) through S private ring slots: lane 0 issues the TMA loads
 //    of a tile (16 rows of K and of V for one page and head, 128-byte
@@ -43,7 +47,7 @@
 
 namespace kvq {
 
-// Largest batch the decode kernels accept (the unit prefix lives in shared memory).
+// Largest batch the decode kernels accept (three per-sequence arrays live in shared memory).
 constexpr int32_t kGqaMaxBatch = 8000;   // three [B+1] arrays in shared memory
 
 // ---------------------------------------------------------------------------
