@@ -23,14 +23,16 @@
 //    E4M3 subnormal step 2^-9 (at most 2^-10 away, against a row maximum of
 //    at least 128).  A pre-pass writes both terms of every (sequence, 64-head
 //    half) as the shared-memory image the MMAs read.
-//  * One thread issues a tcgen05.mma only about every 55 cycles, and an
-//    M=128 (64 rows per SM), N=64, K=32 E4M3 MMA uses the tensor core
-//    poorly unless several are in flight.  So two warps issue: stream k
-//    takes every other 32-dim K-step of QK^T (both query terms) into its
-//    own S accumulator (three per stream, so QK^T runs two blocks ahead),
-//    then PV of the block two back for value-dim half k (N = 256).  The
-//    softmax adds the partial scores; the fixed order per stream keeps PV,
-//    which frees the P and V buffers, from queuing behind QK^T.
+//  * MMA issue: one warp issues every QK^T (18 K-steps of 32 dims, both
+//    query terms, into one of three S accumulators, so it runs up to three
+//    blocks ahead of the softmax) and another every PV (both value-dim
+//    halves, N = 256 each), each in block order.  Each runs its loop as a
+//    whole warp with warp-uniform operands (descriptors from the
+//    shared-memory base, the constant tensor-memory base, the block
+//    counters) and one lane chosen by elect.sync issues: a lane issuing
+//    from divergent code takes about a hundred cycles per MMA, a warp with
+//    uniform operands a few tens, close to the pipe's own rate for these
+//    shapes.
 //  * PV: kind::f8f6f4 as well, on the stored value codes.  P, with the
 //    token's scale folded in and a per-head power of two 2^f, is split into
 //    three E4M3 terms (t0 = E4M3(v), t1 = E4M3(v - t0), t2 = E4M3(v - t0 -
@@ -51,12 +53,15 @@
 //    warps holding the same 32 heads exchange partial maxima and sums
 //    through shared memory.  Scores are scaled to base 2 and exponentiated
 //    against a reference max that moves only when a score exceeds it by 2^8
-//    (then O is rescaled in TMEM).
+//    (then O is rescaled in TMEM).  A block's token scales are read before
+//    its S is waited for, and a rescale of O waits for the previous block's
+//    PV only after this block's P is stored, so that wait overlaps the P
+//    terms.
 //  * Warp roles per CTA: 0 TMA producer (five key stages, page ids read 32
-//    blocks ahead); 1-2 MMA streams (leader CTA only; warp 1 also owns the
-//    tensor memory); 3-10 softmax, P and O read-out; 11 token scales for the
-//    softmax and the value copies.  S has three buffers per MMA stream; V
-//    and P two each, freed by the completion of the PV that read them.
+//    blocks ahead); 1 QK^T and 2 PV issue (leader CTA only; warp 1 also owns
+//    the tensor memory); 3-10 softmax, P and O read-out; 11 token scales for
+//    the softmax and the value copies.  S has three buffers; V and P two
+//    each, freed by the completion of the PV that read them.
 //  * Work split as in the 8-head kernel: the pre-pass also writes the prefix
 //    of 64-token blocks over the sequences, the blocks of all sequences are
 //    split evenly over the CTA pairs (split-KV), each pair writes one
@@ -76,13 +81,8 @@ constexpr int kH = 64;     // heads per CTA
 constexpr int kDk = 576;
 constexpr int kDv = 512;
 constexpr int kBlk = 64;   // tokens per block
-#ifndef KVQ_WIDE_STREAMS
-#define KVQ_WIDE_STREAMS 2
-#endif
-constexpr int kNumMma = KVQ_WIDE_STREAMS;             // MMA streams (2 or 4)
-static_assert(kNumMma == 2 || kNumMma == 4, "MMA streams");
-constexpr int kWarpMma = 1;                           // warps 1 .. kNumMma
-constexpr int kWarpSoftmax = kWarpMma + kNumMma;      // 8 softmax warps
+constexpr int kWarpMma = 1;                           // warp 1 QK^T, warp 2 PV
+constexpr int kWarpSoftmax = kWarpMma + 2;            // 8 softmax warps
 constexpr int kWarpV = kWarpSoftmax + 8;              // scales and value copies
 constexpr int kThreads = 32 * (kWarpV + 1);
 
@@ -99,7 +99,7 @@ constexpr int kPTerm = kH * kBlk;                     // one term: 64 heads x 64
 constexpr int kPBuf = kPTerms * kPTerm;
 constexpr int kNSc = 4;                               // scale ring entries
 constexpr int kNP = 2;                                // P buffers (freed with V: kPvDone)
-constexpr int kNS = 3;                                // S buffers per MMA stream
+constexpr int kNS = 3;                                // S buffers
 
 constexpr int kOffQ = 0;
 constexpr int kOffK = 74752;                          // kQImage rounded up to 1 KB
@@ -131,7 +131,7 @@ enum {
   kQFull = kScR + kNSc,
   kVFull = kQFull + 1,
   kDrain = kVFull + 2,
-  kNumBars = kDrain + 4
+  kNumBars = kDrain + 2
 };
 constexpr int kOffTmem = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = 1024 + kOffTmem + 16;
@@ -139,10 +139,15 @@ static_assert(kQImage <= kOffK, "query image overlaps the key stages");
 static_assert(kNK <= 8, "stage flags");
 static_assert(kSmemBytes <= 232448, "shared memory");
 
-// TMEM columns: O at [0, 256) (value-dim half h of the pair at 128*h), the
-// S accumulator of MMA stream k, buffer s, at 256 + 32*(kNS*k + s).
-static_assert(256 + 32 * kNS * kNumMma <= 512, "tensor memory");
+// TMEM columns: O at [0, 256) (value-dim half h of the pair at 128*h), S
+// buffer s at 256 + 32*s.
+static_assert(256 + 32 * kNS <= 512, "tensor memory");
 constexpr uint32_t kTmemCols = 512;
+// The kernel allocates all 512 columns, so the allocation starts at lane 0,
+// column 0: the MMA warps address tensor memory from this constant (a
+// uniform operand), and a pair whose allocation reports another address
+// records kErrTmemBase and does no work.
+constexpr uint32_t kTmemBase = 0;
 constexpr uint32_t kColS = 256;
 
 // Instruction descriptors (kind::f8f6f4, E4M3 x E4M3): FP32 accumulate
@@ -337,31 +342,93 @@ __device__ __forceinline__ void for_pieces(const Params& p, int32_t u0, int32_t 
   }
 }
 
-// Stream k's share of QK^T for one block: K-steps (32 dims each) k,
-// k + kNumMma, ... of the 18, each as two MMAs (the hi and the lo query
-// term) into the stream's own S accumulator.  Each descriptor is a base plus a
-// constant in its address field (addresses stay below 256 KB, so the
-// 14-bit field cannot carry).
-__device__ __forceinline__ void issue_qk(uint32_t d, uint32_t sq, uint32_t sk, int k) {
-  const uint64_t qa = smem_desc(sq, 16, 1024, 2), ka = smem_desc(sk, 16, 1024, 2);
-  const uint64_t qt = smem_desc(sq + 4 * kQAtom, 16, 512, 4);
-  const uint64_t kt = smem_desc(sk + 4 * kQkAtom, 16, 512, 4);
+// A bounded wait whose result is the same for every lane of the warp.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity));
+}
+
+// Two MMA warps of the leader CTA: one issues QK^T of every block (18
+// K-steps x 2 query terms into one S accumulator), the other PV of every
+// block for both value-dim halves, each in block order.  Each runs its loop
+// as a whole warp with warp-uniform operands (descriptors from the
+// shared-memory base, the constant tensor-memory base, the block counters)
+// and one elected lane issues each tcgen05 instruction.
+__device__ __forceinline__ void qk_warp(const Params& p, uint8_t* smem, uint64_t* bars,
+                                        int32_t u0, int32_t u1) {
+  const uint32_t sq = smem_u32(smem + kOffQ), sk = smem_u32(smem + kOffK);
   constexpr uint64_t kLo = kQPart >> 4;                // the lo term, as a descriptor offset
+  int32_t j = 0, item = 0;
+  bool ok = true;
+  for_pieces(p, u0, u1, [&](int, int32_t, int32_t nt) {
+    ok = ok && wait_bar_warp(&bars[kQReady], item & 1);
+    for (int32_t i = 0; i < nt && ok; ++i, ++j) {
+      const int s = j % kNK, s3 = j % kNS;
+      ok = wait_bar_warp(&bars[kKFull + s], static_cast<uint32_t>(j / kNK) & 1u);
+      if (ok && j >= kNS)
+        ok = wait_bar_warp(&bars[kSFree + s3], static_cast<uint32_t>((j / kNS) & 1) ^ 1u);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t d = kTmemBase + kColS + 32 * s3;
+      const uint32_t sks = sk + s * kStage;
+      const uint64_t qa = smem_desc(sq, 16, 1024, 2), ka = smem_desc(sks, 16, 1024, 2);
+      const uint64_t qt = smem_desc(sq + 4 * kQAtom, 16, 512, 4);
+      const uint64_t kt = smem_desc(sks + 4 * kQkAtom, 16, 512, 4);
 #pragma unroll
-  for (int t = 0; t < (18 + kNumMma - 1) / kNumMma; ++t) {
-    const int ks = k + kNumMma * t;
-    if (ks < 16) {                           // dims 0..511: 128-byte-swizzled atoms
-      const uint64_t qo = qa + (((ks >> 2) * kQAtom + (ks & 3) * 32) >> 4);
-      const uint64_t ko = ka + (((ks >> 2) * kQkAtom + (ks & 3) * 32) >> 4);
-      umma_pair_f8(d, qo, ko, kIdescQK, t > 0 ? 1u : 0u);
-      umma_pair_f8(d, qo + kLo, ko, kIdescQK, 1u);
-    } else if (ks < 18) {                    // dims 512..575: the 64-byte-swizzled tail
-      const uint64_t qo = qt + (((ks - 16) * 32) >> 4);
-      const uint64_t ko = kt + (((ks - 16) * 32) >> 4);
-      umma_pair_f8(d, qo, ko, kIdescQK, 1u);
-      umma_pair_f8(d, qo + kLo, ko, kIdescQK, 1u);
+      for (int ks = 0; ks < 16; ++ks) {          // dims 0..511: 128-byte-swizzled atoms
+        const uint64_t qo = qa + (((ks >> 2) * kQAtom + (ks & 3) * 32) >> 4);
+        const uint64_t ko = ka + (((ks >> 2) * kQkAtom + (ks & 3) * 32) >> 4);
+        umma_pair_f8_warp(d, qo, ko, kIdescQK, ks > 0 ? 1u : 0u);
+        umma_pair_f8_warp(d, qo + kLo, ko, kIdescQK, 1u);
+      }
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {           // dims 512..575: the 64-byte-swizzled tail
+        umma_pair_f8_warp(d, qt + ((ks * 32) >> 4), kt + ((ks * 32) >> 4), kIdescQK, 1u);
+        umma_pair_f8_warp(d, qt + ((ks * 32) >> 4) + kLo, kt + ((ks * 32) >> 4), kIdescQK, 1u);
+      }
+      umma_commit_pair_warp(&bars[kSFull + s3]);
+      umma_commit_pair_warp(&bars[kKFree + s]);
     }
-  }
+    ++item;
+  });
+  umma_commit_pair_local_warp(&bars[kDrain]);
+  mbar_wait_cluster(&bars[kDrain], 0);
+}
+
+__device__ __forceinline__ void pv_warp(const Params& p, uint8_t* smem, uint64_t* bars,
+                                        int32_t u0, int32_t u1) {
+  const uint32_t sv = smem_u32(smem + kOffV), sp = smem_u32(smem + kOffP);
+  int32_t j = 0, item = 0;
+  bool ok = true;
+  for_pieces(p, u0, u1, [&](int, int32_t, int32_t nt) {
+    for (int32_t i = 0; i < nt && ok; ++i, ++j) {
+      const int x = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      ok = wait_bar_warp(&bars[kPReady + x], ph) && wait_bar_warp(&bars[kVReady + x], ph);
+      // O must be free of the previous piece's epilogue
+      if (ok && i == 0 && item > 0) ok = wait_bar_warp(&bars[kOFree], (item - 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      // A: P, one K-major tile per term (rows of 64 token codes, 64-byte
+      // swizzle); B: the value codes, MN-major, 8-token groups of 1 KB;
+      // value half h into O columns [128h, 128h + 128)
+      const uint64_t pa = smem_desc(sp + (j % kNP) * kPBuf, 16, 512, 4);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint64_t va = smem_desc(sv + x * kVBuf + h * kVHalf, kVHalf, 1024, 2);
+#pragma unroll
+        for (int ks = 0; ks < kBlk / 32; ++ks)
+#pragma unroll
+          for (int t = 0; t < kPTerms; ++t)
+            umma_pair_f8_warp(kTmemBase + 128 * h, pa + ((t * kPTerm + 32 * ks) >> 4),
+                              va + ((ks * 4096) >> 4), kIdescPV,
+                              (i == 0 && ks == 0 && t == 0) ? 0u : 1u);
+      }
+      umma_commit_pair_warp(&bars[kPvDone + x]);   // frees V buffer x and P buffer j % 2
+    }
+    ++item;
+  });
+  umma_commit_pair_local_warp(&bars[kDrain + 1]);
+  mbar_wait_cluster(&bars[kDrain + 1], 0);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -379,25 +446,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNK; ++s) {
       mbar_init(&bars[kKFull + s], 1);
-      mbar_init(&bars[kKFree + s], kNumMma + 2);   // the MMA streams + both CTAs' V warps
+      mbar_init(&bars[kKFree + s], 3);   // the QK^T warp's commit + both CTAs' V warps
       mbar_init(&bars[kKPeerFull + s], 1);
       mbar_init(&bars[kScL + s], 1);
     }
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&bars[kSFree + s], 16);       // per softmax warp, both CTAs
-      mbar_init(&bars[kSFull + s], kNumMma);  // one commit per MMA stream
+      mbar_init(&bars[kSFull + s], 1);   // the QK^T warp's commit
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[kPReady + s], 16);
       mbar_init(&bars[kVReady + s], 2);         // one V warp per CTA
-      mbar_init(&bars[kPvDone + s], kNumMma);
+      mbar_init(&bars[kPvDone + s], 1);  // the PV warp's commit
       mbar_init(&bars[kVFull + s], 1);          // plus 16 KB of copies
     }
     for (int s = 0; s < kNSc; ++s) mbar_init(&bars[kScR + s], 1);
     mbar_init(&bars[kQReady], 2);
     mbar_init(&bars[kOFree], 16);
     mbar_init(&bars[kQFull], 1);
-    for (int s = 0; s < kNumMma; ++s) mbar_init(&bars[kDrain + s], 1);
+    for (int s = 0; s < 2; ++s) mbar_init(&bars[kDrain + s], 1);
     fence_barrier_init();
   }
   if (warp == kWarpMma) {
@@ -418,7 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // get an empty range and only set up and tear down.
   const int64_t U = __ldg(p.ws_pre + p.B);
   const int64_t N = working_ctas(p.num_pairs, U, 1);     // min(pairs, U)
-  const bool works = pair < N;
+  if (tbase != kTmemBase && threadIdx.x == 0) atomicOr(&g_error_flags, kErrTmemBase);
+  const bool works = pair < N && tbase == kTmemBase;
   const int32_t u0 = works ? static_cast<int32_t>(U * pair / N) : 0;
   const int32_t u1 = works ? static_cast<int32_t>(U * (pair + 1) / N) : 0;
   const int32_t nblk = u1 - u0;
@@ -487,69 +555,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_cluster(&bars[kScL + j % kNK], ph);
       }
     }
-  } else if (warp < kWarpMma + kNumMma) {
-    // ---------------- MMA issue, kNumMma streams (leader CTA) ----------------
-    // Stream k issues its share of QK^T for block j, then (streams 0 and 1)
-    // PV of block j-1 for value-dim half k.  A thread issues a
-    // tcgen05.mma only about every 55 cycles, so several streams keep the
-    // tensor core fed; the fixed order per stream keeps PV (which frees the
-    // P and V buffers) from queuing behind QK^T.
-    if (rank == 0 && lane == 0) {
-      const int k = warp - kWarpMma;
-      const uint32_t sq = smem_u32(smem + kOffQ), sk = smem_u32(smem + kOffK);
-      const uint32_t sv = smem_u32(smem + kOffV), sp = smem_u32(smem + kOffP);
-      const uint32_t dcol = tbase + kColS + 32 * kNS * k;
-      int32_t j = 0, item = 0;
-      bool ok = true;
-      // PV of block jj, value-dim half h = k (dims 256h + [0, 256) across
-      // the pair) into O columns [128h, 128h + 128); streams 2, 3 have none
-      auto pv = [&](int32_t jj, bool first) {
-        const int x = jj & 1;
-        const uint32_t ph = (jj >> 1) & 1;
-        ok = ok && wait_bar(&bars[kPReady + x], ph) && wait_bar(&bars[kVReady + x], ph);
-        if (ok && first && item > 0) ok = wait_bar(&bars[kOFree], (item - 1) & 1);
-        if (!ok) return;
-        tc_fence_after();
-        // A: P, one K-major tile per term (rows of 64 token codes, 64-byte
-        // swizzle); B: the value codes, MN-major, 8-token groups of 1 KB
-        const uint64_t pa = smem_desc(sp + (jj % kNP) * kPBuf, 16, 512, 4);
-        if (k < 2) {
-          const uint64_t va = smem_desc(sv + x * kVBuf + k * kVHalf, kVHalf, 1024, 2);
-#pragma unroll
-          for (int ks = 0; ks < kBlk / 32; ++ks)
-#pragma unroll
-            for (int t = 0; t < kPTerms; ++t)
-              umma_pair_f8(tbase + 128 * k, pa + ((t * kPTerm + 32 * ks) >> 4),
-                           va + ((ks * 4096) >> 4), kIdescPV,
-                           (first && ks == 0 && t == 0) ? 0u : 1u);
-        }
-        umma_commit_pair(&bars[kPvDone + x]);   // frees V buffer x and P buffer jj % 2
-      };
-      // Within a piece QK^T runs two blocks ahead of PV (three S buffers):
-      // QK(j), then PV(j-2); the piece's last two PVs are issued before the
-      // next piece's QK^T, which waits for its query image, loaded only
-      // once the softmax has finished this piece.
-      for_pieces(p, u0, u1, [&](int, int32_t, int32_t nt) {
-        ok = ok && wait_bar(&bars[kQReady], item & 1);
-        for (int32_t i = 0; i < nt && ok; ++i, ++j) {
-          const int s = j % kNK, s3 = j % kNS;
-          ok = wait_bar(&bars[kKFull + s], static_cast<uint32_t>(j / kNK) & 1u);
-          if (ok && j >= kNS)
-            ok = wait_bar(&bars[kSFree + s3], static_cast<uint32_t>((j / kNS) & 1) ^ 1u);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(dcol + 32 * s3, sq, sk + s * kStage, k);
-          umma_commit_pair(&bars[kSFull + s3]);
-          umma_commit_pair(&bars[kKFree + s]);
-          if (i >= 2) pv(j - 2, i == 2);
-        }
-        if (ok)
-          for (int32_t r = nt >= 2 ? nt - 2 : 0; r < nt; ++r) pv(j - nt + r, r == 0);
-        ++item;
-      });
-      // every MMA issued has finished before either CTA leaves
-      umma_commit_pair_local(&bars[kDrain + k]);
-      mbar_wait_cluster(&bars[kDrain + k], 0);
+  } else if (warp < kWarpSoftmax) {
+    // ---------------- MMA issue (leader CTA): QK^T warp, PV warp ----------------
+    if (rank == 0) {
+      if (warp == kWarpMma) qk_warp(p, smem, bars, u0, u1);
+      else pv_warp(p, smem, bars, u0, u1);
     }
   } else if (warp == kWarpV) {
     // ---------------- token scales and value copies ----------------
@@ -681,31 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int32_t i = 0; i < nt; ++i, ++j) {
         const int s2 = j & 1, s3 = j % kNS;
         const int32_t nvalid = min(kBlk, ntok - (t0 + i) * kBlk);
-        ok = ok && wait_bar(&bars[kSFull + s3], static_cast<uint32_t>(j / kNS) & 1u);
         ok = ok && wait_bar(&bars[kScR + (j & (kNSc - 1))], (j >> 2) & 1);
-        ok = __all_sync(0xffffffffu, ok);                   // tcgen05.ld is warp-collective
-        tc_fence_after();
-        // the streams' partial scores (each covers its share of the dims)
-        float sacc[16];
-        if (ok) {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) sacc[c] = 0.0f;
-#pragma unroll
-          for (int k2 = 0; k2 < kNumMma; k2 += 2) {
-            uint32_t r0[16], r1[16];
-            tmem_ld16(tl + kColS + 32 * (kNS * k2 + s3) + 16 * ch, r0);
-            tmem_ld16(tl + kColS + 32 * (kNS * (k2 + 1) + s3) + 16 * ch, r1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) sacc[c] += __uint_as_float(r0[c]) + __uint_as_float(r1[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) sacc[c] = 0.0f;
-        }
-        tc_fence_before();
-        // this thread's 16 token scales (0 past the end of the sequence or off
-        // the cache) and the block's largest scale
         float sc[16];
         const float smax = ring_max[j & (kNSc - 1)];
         {
@@ -719,6 +705,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             sc[4 * k + 3] = v.w;
           }
         }
+        ok = ok && wait_bar(&bars[kSFull + s3], static_cast<uint32_t>(j / kNS) & 1u);
+        ok = __all_sync(0xffffffffu, ok);                   // tcgen05.ld is warp-collective
+        tc_fence_after();
+        // the block's scores
+        float sacc[16];
+        if (ok) {
+          uint32_t r0[16];
+          tmem_ld16(tl + kColS + 32 * s3 + 16 * ch, r0);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) sacc[c] = __uint_as_float(r0[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) sacc[c] = 0.0f;
+        }
+        tc_fence_before();
+        // this thread's 16 token scales (0 past the end of the sequence or off
+        // the cache) and the block's largest scale
         float x[16];
         float bm = kNegInf;
 #pragma unroll
@@ -751,29 +755,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float vb = ex2(bm - m_new) * smax;
         int f_new = f_p;
         if (vb > 0.0f && (!f_set || vb * pow2f(f_p) > 448.0f)) f_new = pow2_exponent(vb);
-        if (__any_sync(0xffffffffu, m_new != m_ref || f_new != f_p)) {
+        const bool rescale = __any_sync(0xffffffffu, m_new != m_ref || f_new != f_p);
+        float r = 1.0f;
+        if (rescale) {
           const float rm = ex2(m_ref - m_new);            // 0 on the first block, 1 if unmoved
           // before f is first set every P was 0, so O needs no power-of-two factor
-          const float r = f_set ? rm * pow2f(f_new) * pow2f(-f_p) : rm;
+          r = f_set ? rm * pow2f(f_new) * pow2f(-f_p) : rm;
           l_part *= rm;
-          if (i > 0) {
-            // O must not be in use by the previous block's PV
-            ok = ok && wait_bar(&bars[kPvDone + ((j - 1) & 1)], ((j - 1) >> 1) & 1);
-            ok = __all_sync(0xffffffffu, ok);
-            tc_fence_after();
-            if (ok) {                                     // this warp's half of O's columns
-#pragma unroll 1
-              for (int cc = 4 * ch; cc < 4 * ch + 4; ++cc) {
-                uint32_t o[32];
-                tmem_ld32(tl + 32 * cc, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * r);
-                tmem_st32(tl + 32 * cc, o);
-              }
-              tmem_wait_st();
-            }
-          }
         }
         m_ref = m_new;
         f_p = f_new;
@@ -807,6 +795,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < kPTerms; ++t)
             *reinterpret_cast<uint4*>(pbuf + t * kPTerm + sw64(hl, part)) =
                 make_uint4(pt[t][0], pt[t][1], pt[t][2], pt[t][3]);
+        }
+        if (rescale && i > 0) {
+          // O rescale, after P(j) is stored: O must not be in use by PV(j-1)
+          ok = ok && wait_bar(&bars[kPvDone + ((j - 1) & 1)], ((j - 1) >> 1) & 1);
+          ok = __all_sync(0xffffffffu, ok);
+          tc_fence_after();
+          if (ok) {                                       // this warp's half of O's columns
+#pragma unroll 1
+            for (int cc = 4 * ch; cc < 4 * ch + 4; ++cc) {
+              uint32_t o[32];
+              tmem_ld32(tl + 32 * cc, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * r);
+              tmem_st32(tl + 32 * cc, o);
+            }
+            tmem_wait_st();
+          }
         }
         tc_fence_before();
         fence_proxy_async_smem();

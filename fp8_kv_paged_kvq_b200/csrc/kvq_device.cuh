@@ -15,6 +15,7 @@ namespace kvq {
 // one translation unit, so this definition appears once.
 __device__ uint32_t g_error_flags = 0;
 constexpr uint32_t kErrWaitTimeout = 1u;
+constexpr uint32_t kErrTmemBase = 2u;   // a full tensor-memory allocation did not start at 0
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -411,6 +412,23 @@ __device__ __forceinline__ void umma_pair_f16(uint32_t d_tmem, uint64_t a_desc, 
       : "memory");
 }
 
+// The same MMA for a whole warp: every lane passes the same (warp-uniform)
+// operands and one lane, chosen by elect.sync, issues it.  With operands
+// the compiler keeps in uniform registers a warp issues an MMA every few
+// tens of cycles; one lane in divergent code takes about a hundred.
+__device__ __forceinline__ void umma_pair_f8_warp(uint32_t d_tmem, uint64_t a_desc,
+                                                  uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;"
+      "\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on the mbarrier at the same offset in both CTAs of the pair once all
 // earlier tcgen05 operations of this thread have completed.
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
@@ -453,11 +471,33 @@ __device__ __forceinline__ uint4 ld_cluster128(uint32_t addr) {
   return v;
 }
 
+// umma_commit_pair for a whole warp (the lane elect.sync picks, the same
+// lane that issued the warp's MMAs, commits).
+__device__ __forceinline__ void umma_commit_pair_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+
 // Same, arriving only on this CTA's barrier.
 __device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// umma_commit_pair_local for a whole warp.
+__device__ __forceinline__ void umma_commit_pair_local_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
 }
 
 // 32 consecutive 32-bit columns of this thread's TMEM lane.

@@ -307,7 +307,10 @@ kvq_status kvq_e4m3_quantize_bits(uint32_t start, uint32_t count, float scale, u
  * early, so that launch's outputs are invalid), or, in kvq_validate, a
  * failing CTA's wait for the clean result of the same call (the mask bytes
  * written after it may then be overwritten by that late clean result, so
- * the call's outputs are invalid).  *flags_host receives the word.
+ * the call's outputs are invalid).  Bit 1: the wide-group decode kernel's
+ * tensor-memory allocation (all 512 columns, so it starts at column 0) came
+ * back at another address; that CTA pair did no work and the call's outputs
+ * are invalid.  *flags_host receives the word.
  */
 kvq_status kvq_device_error(uint32_t* flags_host);
 
