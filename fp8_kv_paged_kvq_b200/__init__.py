@@ -26,6 +26,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = range(5)
+# bits of the device-side error word (kvq_device_error)
+DEVICE_ERR_WAIT_TIMEOUT = 1    # a bounded wait gave up: that launch's outputs are invalid
+DEVICE_ERR_TMEM_BASE = 2       # a wide-kernel pair's tensor memory was not at column 0
 FP8_E4M3, BF16 = 0, 1
 SCALE_TENSOR, SCALE_HEAD, SCALE_TOKEN = 0, 1, 2
 
@@ -283,6 +286,7 @@ def wait_timeout_check(timed_out: torch.Tensor, stream=None) -> None:
 
 
 def device_error() -> int:
+    """Read and clear the device-side error word (DEVICE_ERR_* bits)."""
     v = ctypes.c_uint32(0)
     _check("kvq_device_error", lib().kvq_device_error(ctypes.byref(v)))
     return int(v.value)
